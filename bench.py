@@ -1,0 +1,416 @@
+"""Benchmark of the block-sparse video self-attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload h3_768p_5s] [--top-k K] [--no-cpu-baseline] [--no-e2e]
+
+One step = one whole attention call (pool -> summarize -> select -> attend,
+all through the C ABI) over one batch of synthetic bf16 input of the 768p-5s
+H3 shape (B=1, H=56, N=37,740, d=128, top_k=64, anchor-weighted summaries).
+Prints ONE JSON line on rank 0.  Multi-GPU (torchrun): every rank runs its own
+independent call on its own inputs (weak scaling, no data-path collective);
+the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/attention call and effective TFLOP/s vs bf16 peak (56 heads, d=128, top_k=64)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="h3_768p_5s")
+    ap.add_argument("--top-k", type=int, default=None)
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override H (small profiling captures only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ accounting
+
+def block_sizes(N):
+    nb = -(-N // 128)
+    sizes = np.full(nb, 128, dtype=np.int64)
+    sizes[-1] = N - 128 * (nb - 1)
+    return sizes
+
+
+def effective_pairs(idx, cnt, N, prefix):
+    """Computed (query, key or summary) pairs of all heads: exact pairs over
+    the real tokens of each listed block plus one summary column per skipped
+    video block for every video query row (masked columns excluded)."""
+    sizes = block_sizes(N)
+    nb = len(sizes)
+    pb = prefix // 128
+    idx = idx.reshape(-1, nb, idx.shape[-1])
+    cnt = cnt.reshape(-1, nb)
+    valid = np.arange(idx.shape[-1])[None, None, :] < cnt[:, :, None]
+    exact = np.where(valid, sizes[np.clip(idx, 0, nb - 1)], 0).sum(-1)
+    summ = np.where(np.arange(nb)[None, :] >= pb, (nb - pb) - (cnt - pb), 0)
+    return int((sizes[None, :] * (exact + summ)).sum())
+
+
+def stage_bytes(B, H, N, nb, kcap):
+    """Algorithmic HBM bytes of the pool + summarize passes (read Q, K, V once;
+    write qpool, kpool fp32, k~, v~ bf16, bias, anchor)."""
+    bh = B * H
+    reads = 3 * bh * N * 128 * 2
+    writes = bh * nb * 128 * (4 + 4 + 2 + 2) + bh * nb * 4 + bh * 128 * 4
+    return reads + writes
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3):
+    """The fp64 oracle as it stands, on whole heads, until ~budget_s of CPU work."""
+    import oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    pairs = 0
+    t0 = time.perf_counter()
+    heads = 0
+    for h in range(min(max_heads, len(Qh))):
+        out = orc.forward_head(Qh[h], Kh[h], Vh[h], cfg["top_k"], cfg["prefix"], cfg["variant"])
+        pairs += orc.effective_pairs(len(Qh[h]), out["lists"], cfg["prefix"] // 128)
+        heads += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = 4 * 128 * pairs
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{heads} of {cfg['H']} heads of the workload, whole path per head "
+                      f"(numpy fp64, BLAS threads = {cores}); {dt:.1f} s, "
+                      f"{dt / heads:.2f} s/head"}, dt / heads
+
+
+def run_reference(args, cfg):
+    """Reference arm: the fp64 CPU oracle timed on the host cores, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    from block_sparse_video_bsa_b200.inputs import make_tensor
+    # one head of the workload per step (bounded sample), inputs built on the CPU
+    B, H, N = cfg["B"], cfg["H"], cfg["N"]
+    heads = [make_tensor(t, 1, 1, N, 128, cfg["kind"], seed=0, device="cpu")[0, 0]
+             .double().numpy() for t in ("q", "k", "v")]
+    import oracle as orc
+    times, pairs_l = [], []
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        out = orc.forward_head(heads[0], heads[1], heads[2], cfg["top_k"], cfg["prefix"],
+                               cfg["variant"])
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            pairs_l.append(orc.effective_pairs(N, out["lists"], cfg["prefix"] // 128))
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    ms = 1e3 * sum(times) / len(times)
+    value = 4 * 128 * sum(pairs_l) / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_block(cfg, sample="1 of 56 heads per step"),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "one whole head (of 56) of the workload per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_block(cfg, **extra):
+    d = {"workload": cfg["name"], "B": cfg["B"], "H": cfg["H"], "N": cfg["N"], "d": 128,
+         "top_k": cfg["top_k"], "prefix": cfg["prefix"], "summary": cfg["variant"],
+         "inputs": cfg["kind"], "l2": "inputs larger than L2 (Q+K+V = "
+         f"{3 * cfg['B'] * cfg['H'] * cfg['N'] * 256 / 1e9:.2f} GB per step)"}
+    d.update(extra)
+    return d
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    args = parse_args()
+    from block_sparse_video_bsa_b200.inputs import CONFIGS
+    cfg = dict(CONFIGS[args.workload])
+    cfg["name"] = args.workload
+    if args.top_k is not None:
+        cfg["top_k"] = args.top_k
+    if args.heads is not None:
+        cfg["H"] = args.heads
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from block_sparse_video_bsa_b200 import bsa
+    from block_sparse_video_bsa_b200.inputs import make_qkv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    B, H, N = cfg["B"], cfg["H"], cfg["N"]
+    top_k, prefix, variant = cfg["top_k"], cfg["prefix"], cfg["variant"]
+    Q, K, V = make_qkv(B, H, N, 128, cfg["kind"], seed=rank, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    p = bsa.params(B, H, N, top_k, prefix, variant, dev_status=status)
+    buf = bsa.stage_buffers(B, H, N, top_k, prefix, variant, device=dev)
+    O = torch.empty_like(Q)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        bsa.bsa_pool(p, Q, buf["qpool"], buf["anchor"], stream)
+        if ev:
+            ev[1].record(stream)
+        bsa.bsa_summarize(p, K, V, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"],
+                          buf["bias"], stream)
+        if ev:
+            ev[2].record(stream)
+        bsa.bsa_select(p, buf["qpool"], buf["kpool"], buf["idx"], buf["cnt"], stream)
+        if ev:
+            ev[3].record(stream)
+        bsa.bsa_attend(p, Q, K, V, buf["idx"], buf["cnt"], buf["ksum"], buf["vsum"], buf["bias"],
+                       O, None, stream)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {bsa.status_string(int(status.item()))}")
+    pairs = effective_pairs(buf["idx"].cpu().numpy(), buf["cnt"].cpu().numpy(), N, prefix) \
+        * 1  # all B*H heads
+    flops_step = 4 * 128 * pairs
+    nb = bsa.bsa_num_blocks(p)
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)   # let the sampler start before the timed region
+    for s in range(args.steps):
+        step(events[s])
+    torch.cuda.synchronize(dev)
+    clock_info = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {bsa.status_string(int(status.item()))}")
+
+    total_ms = sum(e[0].elapsed_time(e[4]) for e in events)
+    stage_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in events) for i in range(4)]
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * flops_step * args.steps / (total_ms / 1e3) / 1e12
+
+    # end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
+        hO = torch.empty_like(hQ).pin_memory()
+        ws = bsa.workspace(p, dev)
+        for _ in range(2):
+            bsa.bsa_forward_host(p, hQ, hK, hV, hO, None, Q, K, V, O, None, ws, stream)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            bsa.bsa_forward_host(p, hQ, hK, hV, hO, None, Q, K, V, O, None, ws, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e_ms = float(te.item())
+        e2e = {"value": world * flops_step * args.e2e_steps / (e_ms / 1e3) / 1e12,
+               "unit": "TFLOP/s", "ms_per_call": e_ms / args.e2e_steps,
+               "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
+               "d2h_bytes_per_step": O.numel() * O.element_size(),
+               "path": "bsa_forward_host (pinned host Q/K/V -> device -> host O)"}
+        del hQ, hK, hV, hO
+
+    peaks, peak_src = load_peaks()
+    attend_ms = stage_ms[3]
+    attend_tflops = flops_step / (attend_ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    pool_bytes = stage_bytes(B, H, N, nb, bsa.bsa_select_capacity(p))
+    pool_gbs = pool_bytes / ((stage_ms[0] + stage_ms[1]) / 1e3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        hh = [0, 1, 2]
+        Qh = [Q[0, h].double().cpu().numpy() for h in hh]
+        Kh = [K[0, h].double().cpu().numpy() for h in hh]
+        Vh = [V[0, h].double().cpu().numpy() for h in hh]
+        cpu, _ = time_oracle(Qh, Kh, Vh, cfg)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded per-block-offset bf16 Q/K/V of the H3 768p-5s shape)",
+            "config": config_block(cfg, parallelism=f"{world} independent calls (one per GPU)"),
+            "ms_per_call": ms_per_step,
+            "effective_tflop_per_call": flops_step / 1e12,
+            "stages_ms": {"pool": stage_ms[0], "summarize": stage_ms[1], "select": stage_ms[2],
+                          "attend": stage_ms[3]},
+            "roofline": {"kernel": "attend_kernel", "bound": "tensor", "achieved": attend_tflops,
+                         "peak": peak, "unit": "TFLOP/s", "frac": attend_tflops / peak,
+                         "peak_source": f"{peak_src} bf16 burst",
+                         "traffic": read_traffic(cfg)},
+            "pool_summary": {"bound": "hbm", "achieved": pool_gbs,
+                             "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                             "frac": pool_gbs / float(peaks["hbm_gbs"]),
+                             "bytes_per_call": pool_bytes},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 5 * args.steps,
+            "clocks": clock_info,
+            "context": {"pages_rtx_pro_6000_sparse_ms": 30.7 if cfg["N"] == 37_740 else None},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def read_traffic(cfg):
+    """DRAM bytes per attend launch from the committed ncu summary, if it was
+    taken on the current kernel source and this workload; else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "attend_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for ln in open(path):
+        if "=" in ln and not ln.startswith("#"):
+            k, v = ln.split("=", 1)
+            kv[k.strip()] = v.strip()
+    src = os.path.join(ROOT, "block_sparse_video_bsa_b200", "csrc", "attend.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if kv.get("attend_cu_sha256_16") != h or kv.get("workload") != cfg["name"]:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,206 @@
+"""Thin ctypes binding over libbsa.so (include/bsa.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are torch tensors (device memory + streams); the functions
+keep the C names.  There is no fallback: if libbsa.so is missing or the
+device is not sm_100 the call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbsa.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "bsa.h")
+
+BSA_OK, BSA_ERR_INVALID, BSA_ERR_ALIGN, BSA_ERR_CUDA, BSA_ERR_TIMEOUT, BSA_ERR_UNSUPPORTED = range(6)
+VARIANTS = {"anchor": 0, "mean": 1}
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class bsa_params(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+        ("D", ctypes.c_int32), ("top_k", ctypes.c_int32), ("prefix", ctypes.c_int32),
+        ("variant", ctypes.c_int32), ("dev_status", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+_P = ctypes.POINTER(bsa_params)
+_vp = ctypes.c_void_p
+_SIGS = {
+    "bsa_num_blocks": (ctypes.c_int32, [_P]),
+    "bsa_select_capacity": (ctypes.c_int32, [_P]),
+    "bsa_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "bsa_pool": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp]),
+    "bsa_summarize": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_select": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_attend": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_forward": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "bsa_forward_host": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _vp, ctypes.c_size_t, _vp]),
+    "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "bsa_debug_expired_wait": (ctypes.c_int, [_vp, ctypes.c_uint64, _vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbsa.so once (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m "
+                               "block_sparse_video_bsa_b200.build` first")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of the functions include/bsa.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsa_[a-z_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return lib().bsa_status_string(int(status)).decode()
+
+
+def params(B, H, N, top_k, prefix=0, variant="anchor", D=128, dev_status=None) -> bsa_params:
+    v = VARIANTS[variant] if isinstance(variant, str) else int(variant)
+    ds = None if dev_status is None else dev_status.data_ptr()
+    return bsa_params(B, H, N, D, top_k, prefix, v, ds)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc, where):
+    if rc != BSA_OK:
+        raise BsaError(rc, where)
+
+
+# --------------------------------------------------------------- sizes
+
+def bsa_num_blocks(p: bsa_params) -> int:
+    return lib().bsa_num_blocks(ctypes.byref(p))
+
+
+def bsa_select_capacity(p: bsa_params) -> int:
+    return lib().bsa_select_capacity(ctypes.byref(p))
+
+
+def bsa_workspace_bytes(p: bsa_params) -> int:
+    return lib().bsa_workspace_bytes(ctypes.byref(p))
+
+
+# --------------------------------------------------------------- stages
+
+def bsa_pool(p, Q, qpool, anchor, stream=None):
+    _check(lib().bsa_pool(ctypes.byref(p), _ptr(Q), _ptr(qpool), _ptr(anchor), _stream(stream)),
+           "bsa_pool")
+
+
+def bsa_summarize(p, K, V, anchor, kpool, ksum, vsum, bias, stream=None):
+    _check(lib().bsa_summarize(ctypes.byref(p), _ptr(K), _ptr(V), _ptr(anchor), _ptr(kpool),
+                               _ptr(ksum), _ptr(vsum), _ptr(bias), _stream(stream)),
+           "bsa_summarize")
+
+
+def bsa_select(p, qpool, kpool, idx, cnt, stream=None):
+    _check(lib().bsa_select(ctypes.byref(p), _ptr(qpool), _ptr(kpool), _ptr(idx), _ptr(cnt),
+                            _stream(stream)), "bsa_select")
+
+
+def bsa_attend(p, Q, K, V, idx, cnt, ksum, vsum, bias, O, lse=None, stream=None):
+    _check(lib().bsa_attend(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(cnt),
+                            _ptr(ksum), _ptr(vsum), _ptr(bias), _ptr(O), _ptr(lse),
+                            _stream(stream)), "bsa_attend")
+
+
+def bsa_forward(p, Q, K, V, O, lse, workspace, stream=None):
+    _check(lib().bsa_forward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(stream)), "bsa_forward")
+
+
+def bsa_forward_host(p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, stream=None):
+    _check(lib().bsa_forward_host(ctypes.byref(p), _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hO),
+                                  _ptr(hlse), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dO), _ptr(dlse),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream)), "bsa_forward_host")
+
+
+def bsa_debug_expired_wait(dev_status, timeout_ns: int, stream=None):
+    _check(lib().bsa_debug_expired_wait(_ptr(dev_status), int(timeout_ns), _stream(stream)),
+           "bsa_debug_expired_wait")
+
+
+# --------------------------------------------------------------- allocation helpers
+
+def stage_buffers(B, H, N, top_k, prefix=0, variant="anchor", device="cuda"):
+    """Device tensors for the intermediates of the four stages."""
+    p = params(B, H, N, top_k, prefix, variant)
+    nb = bsa_num_blocks(p)
+    kcap = bsa_select_capacity(p)
+    if nb < 0:
+        raise BsaError(BSA_ERR_INVALID, "stage_buffers")
+    f32, bf16, i32 = torch.float32, torch.bfloat16, torch.int32
+    return dict(
+        qpool=torch.empty(B, H, nb, 128, dtype=f32, device=device),
+        anchor=torch.empty(B, H, 128, dtype=f32, device=device),
+        kpool=torch.empty(B, H, nb, 128, dtype=f32, device=device),
+        ksum=torch.empty(B, H, nb, 128, dtype=bf16, device=device),
+        vsum=torch.empty(B, H, nb, 128, dtype=bf16, device=device),
+        bias=torch.empty(B, H, nb, dtype=f32, device=device),
+        idx=torch.empty(B, H, nb, kcap, dtype=i32, device=device),
+        cnt=torch.empty(B, H, nb, dtype=i32, device=device),
+    )
+
+
+def workspace(p: bsa_params, device="cuda") -> torch.Tensor:
+    n = bsa_workspace_bytes(p)
+    if n == 0:
+        raise BsaError(BSA_ERR_INVALID, "bsa_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def forward(Q, K, V, top_k, prefix=0, variant="anchor", return_lse=False, ws=None, stream=None):
+    """O = block-sparse attention(Q, K, V), bf16 [B, H, N, 128] in and out."""
+    B, H, N, D = Q.shape
+    p = params(B, H, N, top_k, prefix, variant, D=D)
+    O = torch.empty_like(Q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=Q.device) if return_lse else None
+    if ws is None:
+        ws = workspace(p, Q.device)
+    bsa_forward(p, Q, K, V, O, lse, ws, stream)
+    return (O, lse) if return_lse else O
+
+
+def topk_from_density(rho: float, N: int, prefix: int = 0) -> int:
+    """Key-block ratio -> integer top_k = ceil(rho * nbv) (the caller's conversion)."""
+    nbv = -(-N // 128) - prefix // 128
+    return max(1, math.ceil(rho * nbv - 1e-9))

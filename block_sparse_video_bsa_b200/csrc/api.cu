@@ -1,0 +1,301 @@
+// C ABI of libbsa.so (declared in include/bsa.h): argument checks, TMA
+// tensor-map construction and the launches of the four stages.  No memory is
+// allocated here and no state is kept between calls except per-device
+// capability / attribute caches.
+#include <mutex>
+
+#include "bsa.h"
+#include "bsa_kernels.h"
+
+namespace {
+
+using bsa::Shape;
+
+constexpr int kMaxN = 1 << 21;       // nb <= 16384 (bitmap / score tile sizes)
+constexpr int kMaxBH = 65535;        // grid.y limit of the per-block kernels
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int shape_of(const bsa_params* p, Shape* s) {
+  if (!p) return BSA_ERR_INVALID;
+  if (p->D != 128 || p->B < 1 || p->H < 1 || p->N < 1 || p->N > kMaxN) return BSA_ERR_INVALID;
+  if (static_cast<int64_t>(p->B) * p->H > kMaxBH) return BSA_ERR_INVALID;
+  if (p->top_k < 1) return BSA_ERR_INVALID;
+  if (p->prefix < 0 || p->prefix % 128 != 0 || p->prefix >= p->N) return BSA_ERR_INVALID;
+  if (p->variant != BSA_SUMMARY_ANCHOR && p->variant != BSA_SUMMARY_MEAN) return BSA_ERR_INVALID;
+  s->B = p->B;
+  s->H = p->H;
+  s->N = p->N;
+  s->nb = (p->N + 127) / 128;
+  s->pb = p->prefix / 128;
+  s->nbv = s->nb - s->pb;
+  s->k_eff = p->top_k < s->nbv ? p->top_k : s->nbv;
+  s->kcap = p->prefix > 0 ? s->nb : s->pb + s->k_eff;
+  s->variant = p->variant;
+  s->prefix = p->prefix;
+  s->dev_status = p->dev_status;
+  return BSA_OK;
+}
+
+// The kernels use tcgen05 / TMA: sm_100 only.  Cached per device.
+int check_device() {
+  static std::mutex mu;
+  static signed char ok[64];
+  static bool init = false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
+  std::lock_guard<std::mutex> g(mu);
+  if (!init) {
+    for (auto& v : ok) v = -1;
+    init = true;
+  }
+  if (dev >= 64) return BSA_ERR_UNSUPPORTED;
+  if (ok[dev] < 0) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return BSA_ERR_CUDA;
+    ok[dev] = (major == 10) ? 1 : 0;
+  }
+  return ok[dev] ? BSA_OK : BSA_ERR_UNSUPPORTED;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 [BH, rows, 128] viewed as a 3-D tensor; box = 64 columns (128 bytes,
+// one swizzle atom) x 128 rows x 1 head.  Rows past `rows` read as zero.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {128, rows, BH};
+  const cuuint64_t strides[2] = {128 * 2, rows * 128 * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct Workspace {
+  float *qpool, *anchor, *kpool, *bias;
+  void *ksum, *vsum;
+  int32_t *idx, *cnt;
+};
+
+size_t carve(const Shape& s, uint8_t* base, Workspace* w) {
+  const size_t bh = static_cast<size_t>(s.B) * s.H;
+  const size_t blocks = bh * s.nb;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += round256(bytes);
+    return p;
+  };
+  uint8_t* qpool = take(blocks * 128 * 4);
+  uint8_t* anchor = take(bh * 128 * 4);
+  uint8_t* kpool = take(blocks * 128 * 4);
+  uint8_t* ksum = take(blocks * 128 * 2);
+  uint8_t* vsum = take(blocks * 128 * 2);
+  uint8_t* bias = take(blocks * 4);
+  uint8_t* idx = take(blocks * static_cast<size_t>(s.kcap) * 4);
+  uint8_t* cnt = take(blocks * 4);
+  if (w) {
+    w->qpool = reinterpret_cast<float*>(qpool);
+    w->anchor = reinterpret_cast<float*>(anchor);
+    w->kpool = reinterpret_cast<float*>(kpool);
+    w->ksum = ksum;
+    w->vsum = vsum;
+    w->bias = reinterpret_cast<float*>(bias);
+    w->idx = reinterpret_cast<int32_t*>(idx);
+    w->cnt = reinterpret_cast<int32_t*>(cnt);
+  }
+  return off;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+int pool_impl(const Shape& s, const void* Q, float* qpool, float* anchor, cudaStream_t st) {
+  return cuda_status(bsa::launch_pool(s, Q, qpool, anchor, st));
+}
+int summarize_impl(const Shape& s, const void* K, const void* V, const float* anchor, float* kpool,
+                   void* ksum, void* vsum, float* bias, cudaStream_t st) {
+  return cuda_status(bsa::launch_summarize(s, K, V, anchor, kpool, ksum, vsum, bias, st));
+}
+int select_impl(const Shape& s, const float* qpool, const float* kpool, int32_t* idx, int32_t* cnt,
+                cudaStream_t st) {
+  return cuda_status(bsa::launch_select(s, qpool, kpool, idx, cnt, st));
+}
+int attend_impl(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* idx,
+                const int32_t* cnt, const void* ksum, const void* vsum, const float* bias, void* O,
+                float* lse, cudaStream_t st) {
+  bsa::AttendMaps maps;
+  const uint64_t bh = static_cast<uint64_t>(s.B) * s.H;
+  if (!make_map(&maps.q, Q, s.N, bh) || !make_map(&maps.k, K, s.N, bh) ||
+      !make_map(&maps.v, V, s.N, bh) || !make_map(&maps.ks, ksum, s.nb, bh) ||
+      !make_map(&maps.vs, vsum, s.nb, bh))
+    return BSA_ERR_UNSUPPORTED;
+  return cuda_status(bsa::launch_attend(s, maps, idx, cnt, bias, O, lse, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t bsa_num_blocks(const bsa_params* p) {
+  Shape s;
+  return shape_of(p, &s) == BSA_OK ? s.nb : -1;
+}
+
+int32_t bsa_select_capacity(const bsa_params* p) {
+  Shape s;
+  return shape_of(p, &s) == BSA_OK ? s.kcap : -1;
+}
+
+size_t bsa_workspace_bytes(const bsa_params* p) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK) return 0;
+  return carve(s, nullptr, nullptr);
+}
+
+int bsa_pool(const bsa_params* p, const void* Q, float* qpool, float* anchor, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !qpool || !anchor) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(qpool, 16) || !aligned(anchor, 16)) return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return pool_impl(s, Q, qpool, anchor, static_cast<cudaStream_t>(stream));
+}
+
+int bsa_summarize(const bsa_params* p, const void* K, const void* V, const float* anchor,
+                  float* kpool, void* ksum, void* vsum, float* bias, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!K || !V || !kpool || !ksum || !vsum || !bias) return BSA_ERR_INVALID;
+  if (s.variant == BSA_SUMMARY_ANCHOR && !anchor) return BSA_ERR_INVALID;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(kpool, 16) || !aligned(ksum, 16) ||
+      !aligned(vsum, 16) || !aligned(bias, 4) || (anchor && !aligned(anchor, 16)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return summarize_impl(s, K, V, anchor, kpool, ksum, vsum, bias, static_cast<cudaStream_t>(stream));
+}
+
+int bsa_select(const bsa_params* p, const float* qpool, const float* kpool, int32_t* idx,
+               int32_t* cnt, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!qpool || !kpool || !idx || !cnt) return BSA_ERR_INVALID;
+  if (!aligned(qpool, 16) || !aligned(kpool, 16) || !aligned(idx, 4) || !aligned(cnt, 4))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return select_impl(s, qpool, kpool, idx, cnt, static_cast<cudaStream_t>(stream));
+}
+
+int bsa_attend(const bsa_params* p, const void* Q, const void* K, const void* V,
+               const int32_t* idx, const int32_t* cnt, const void* ksum, const void* vsum,
+               const float* bias, void* O, float* lse, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !K || !V || !idx || !cnt || !ksum || !vsum || !bias || !O) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(ksum, 16) ||
+      !aligned(vsum, 16) || !aligned(O, 16) || !aligned(idx, 4) || !aligned(cnt, 4) ||
+      !aligned(bias, 4) || (lse && !aligned(lse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return attend_impl(s, Q, K, V, idx, cnt, ksum, vsum, bias, O, lse,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int bsa_forward(const bsa_params* p, const void* Q, const void* K, const void* V, void* O,
+                float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !workspace) return BSA_ERR_INVALID;
+  if (workspace_bytes < carve(s, nullptr, nullptr)) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
+      !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  Workspace w;
+  carve(s, static_cast<uint8_t*>(workspace), &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = pool_impl(s, Q, w.qpool, w.anchor, st))) return rc;
+  if ((rc = summarize_impl(s, K, V, w.anchor, w.kpool, w.ksum, w.vsum, w.bias, st))) return rc;
+  if ((rc = select_impl(s, w.qpool, w.kpool, w.idx, w.cnt, st))) return rc;
+  return attend_impl(s, Q, K, V, w.idx, w.cnt, w.ksum, w.vsum, w.bias, O, lse, st);
+}
+
+int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK, const void* hV,
+                     void* hO, float* hlse, void* dQ, void* dK, void* dV, void* dO, float* dlse,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!hQ || !hK || !hV || !hO) return BSA_ERR_INVALID;
+  const size_t bytes = static_cast<size_t>(s.B) * s.H * s.N * 128 * 2;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Validate the device side before the first copy so an error enqueues nothing.
+  if (!dQ || !dK || !dV || !dO || !workspace) return BSA_ERR_INVALID;
+  if (workspace_bytes < carve(s, nullptr, nullptr)) return BSA_ERR_INVALID;
+  if (!aligned(dQ, 16) || !aligned(dK, 16) || !aligned(dV, 16) || !aligned(dO, 16) ||
+      !aligned(workspace, 256) || (dlse && !aligned(dlse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  if (cudaMemcpyAsync(dQ, hQ, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(dK, hK, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(dV, hV, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  if ((rc = bsa_forward(p, dQ, dK, dV, dO, dlse, workspace, workspace_bytes, stream))) return rc;
+  if (cudaMemcpyAsync(hO, dO, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return BSA_ERR_CUDA;
+  if (hlse && dlse &&
+      cudaMemcpyAsync(hlse, dlse, static_cast<size_t>(s.B) * s.H * s.N * 4, cudaMemcpyDeviceToHost,
+                      st) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  return BSA_OK;
+}
+
+const char* bsa_status_string(int status) {
+  switch (status) {
+    case BSA_OK: return "ok";
+    case BSA_ERR_INVALID: return "invalid argument";
+    case BSA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case BSA_ERR_CUDA: return "CUDA error";
+    case BSA_ERR_TIMEOUT: return "bounded device wait expired";
+    case BSA_ERR_UNSUPPORTED: return "unsupported device (needs sm_100) or driver";
+    default: return "unknown status";
+  }
+}
+
+int bsa_debug_expired_wait(int32_t* dev_status, uint64_t timeout_ns, void* stream) {
+  if (!dev_status || !aligned(dev_status, 4)) return BSA_ERR_INVALID;
+  if (timeout_ns > 10000000000ull) return BSA_ERR_INVALID;
+  int rc = check_device();
+  if (rc) return rc;
+  return cuda_status(bsa::launch_expired_wait(dev_status, timeout_ns,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,37 @@
+// Host-side launchers of the kernels (internal to libbsa.so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bsa {
+
+struct Shape {
+  int B, H, N;      // D is fixed at 128
+  int nb;           // ceil(N / 128)
+  int pb;           // prefix blocks
+  int nbv;          // nb - pb
+  int k_eff;        // min(top_k, nbv)
+  int kcap;         // idx row length
+  int variant;      // 0 anchor, 1 mean
+  int prefix;       // prefix tokens
+  int* dev_status;  // optional
+};
+
+cudaError_t launch_pool(const Shape& s, const void* Q, float* qpool, float* anchor,
+                        cudaStream_t st);
+cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const float* anchor,
+                             float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st);
+cudaError_t launch_select(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
+                          int32_t* cnt, cudaStream_t st);
+
+struct AttendMaps {
+  CUtensorMap q, k, v, ks, vs;   // bf16, box {64, 128, 1}, 128B swizzle
+};
+cudaError_t launch_attend(const Shape& s, const AttendMaps& maps, const int32_t* idx,
+                          const int32_t* cnt, const float* bias, void* O, float* lse,
+                          cudaStream_t st);
+cudaError_t launch_expired_wait(int32_t* dev_status, uint64_t timeout_ns, cudaStream_t st);
+
+}  // namespace bsa

@@ -1,0 +1,259 @@
+// HBM-bound passes over Q, K, V.
+//
+//  pool_q_kernel       one CTA per (query block, head): reads the block's
+//                      128 x 128 bf16 rows once, writes its fp32 mean (qpool).
+//  anchor_kernel       one CTA per head: q-bar = mean of the video query rows
+//                      ("the mean of the video queries as one anchor per
+//                      head", Spark-H3 page, Spark-Reweight bullet), summed
+//                      from qpool * n_i in a fixed order (deterministic).
+//  summarize_kernel    one CTA per (key block, head): reads the K and V rows
+//                      of the block once and writes the pooled key (kpool,
+//                      used by the block score) and the block's summary row
+//                      k~, v~, bias (the compressed branch, Spark-Reweight
+//                      bullet; mean-pooled variant as the baseline it replaces).
+//
+// Thread layout of the per-block kernels: 256 threads, 16 threads per token
+// row (8 bf16 = one 16-byte load each), 16 rows per pass, 8 passes; every
+// thread keeps its 8 rows in registers, so each byte is read from HBM once.
+#include "bsa_device.cuh"
+#include "bsa_kernels.h"
+
+namespace bsa {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// Rows r = g + 16*it of a block (g = tid / 16), 8 dims (tid % 16) * 8 each.
+__device__ __forceinline__ void load_block_rows(const __nv_bfloat16* base, int n, int g, int c,
+                                                uint4 rows[8]) {
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = g + 16 * it;
+    rows[it] = (r < n) ? ld_stream_v4(base + static_cast<size_t>(r) * kDim + c * 8) : zero;
+  }
+}
+
+// Sum of 8-float vectors over the 16 row groups of the CTA.  Each thread
+// passes its partial for dims [8c, 8c+8); thread d < 128 gets dim d's total.
+// `red` is [8 warps][128] floats of shared memory.  Fixed order: xor-16 pair
+// inside the warp, then warps 0..7 in sequence.
+__device__ __forceinline__ float cta_sum_over_rows(const float part[8], float* red, int c) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float v[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = part[k] + __shfl_xor_sync(0xffffffffu, part[k], 16);
+  if (lane < 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) red[warp * kDim + c * 8 + k] = v[k];
+  }
+  __syncthreads();
+  float s = 0.f;
+  if (threadIdx.x < kDim) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[w * kDim + threadIdx.x];
+  }
+  __syncthreads();
+  return s;
+}
+
+__global__ void __launch_bounds__(kThreads) pool_q_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                          float* __restrict__ qpool, int N,
+                                                          int nb) {
+  __shared__ float red[8 * kDim];
+  const int blk = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  const int row0 = blk * kBlock;
+  const int n = min(kBlock, N - row0);
+  const int g = threadIdx.x >> 4, c = threadIdx.x & 15;
+  uint4 rows[8];
+  load_block_rows(Q + (bh * N + row0) * kDim, n, g, c, rows);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    float f[8];
+    bf16x8_to_f32(rows[it], f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] += f[k];
+  }
+  const float s = cta_sum_over_rows(acc, red, c);
+  if (threadIdx.x < kDim) qpool[(bh * nb + blk) * kDim + threadIdx.x] = s / static_cast<float>(n);
+}
+
+// 1024 threads: 8 groups of 128 dims; group gi sums blocks i = pb+gi, pb+gi+8, ...
+__global__ void __launch_bounds__(1024) anchor_kernel(const float* __restrict__ qpool,
+                                                      float* __restrict__ anchor, int N, int nb,
+                                                      int pb) {
+  __shared__ float part[8][kDim];
+  const size_t bh = blockIdx.x;
+  const int d = threadIdx.x & (kDim - 1), gi = threadIdx.x >> 7;
+  const float* qp = qpool + bh * nb * kDim;
+  float s = 0.f;
+  for (int i = pb + gi; i < nb; i += 8) {
+    const float n_i = static_cast<float>(min(kBlock, N - i * kBlock));
+    s += __ldg(qp + static_cast<size_t>(i) * kDim + d) * n_i;
+  }
+  part[gi][d] = s;
+  __syncthreads();
+  if (gi == 0) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += part[k][d];
+    anchor[bh * kDim + d] = t / static_cast<float>(N - pb * kBlock);
+  }
+}
+
+template <int kVariant>  // 0 = anchor-weighted, 1 = mean-pooled
+__global__ void __launch_bounds__(kThreads) summarize_kernel(
+    const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
+    const float* __restrict__ anchor, float* __restrict__ kpool, __nv_bfloat16* __restrict__ ksum,
+    __nv_bfloat16* __restrict__ vsum, float* __restrict__ bias, int N, int nb, float scale) {
+  __shared__ float red[8 * kDim];
+  __shared__ float xs[kBlock];
+  __shared__ float stat[2];
+  const int blk = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  const int row0 = blk * kBlock;
+  const int n = min(kBlock, N - row0);
+  const int tid = threadIdx.x, g = tid >> 4, c = tid & 15;
+  const int lane = tid & 31, warp = tid >> 5;
+
+  uint4 kr[8], vr[8];
+  load_block_rows(K + (bh * N + row0) * kDim, n, g, c, kr);
+  load_block_rows(V + (bh * N + row0) * kDim, n, g, c, vr);
+
+  float ks[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    float f[8];
+    bf16x8_to_f32(kr[it], f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ks[k] += f[k];
+  }
+
+  float kt[8], vt[8];
+  float lse = 0.f;
+  if (kVariant == 0) {
+    float a[8];
+    const float4* ap = reinterpret_cast<const float4*>(anchor + bh * kDim + c * 8);
+    const float4 a0 = __ldg(ap), a1 = __ldg(ap + 1);
+    a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
+    a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+    // x_r = anchor . k_r * scale for the 8 rows of this thread's group
+    float x[8];
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      float f[8];
+      bf16x8_to_f32(kr[it], f);
+      float p = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) p = fmaf(a[k], f[k], p);
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+      x[it] = p * scale;
+    }
+    if (c == 0) {
+#pragma unroll
+      for (int it = 0; it < 8; ++it) xs[g + 16 * it] = x[it];
+    }
+    __syncthreads();
+    if (warp == 0) {  // block max and log-sum-exp over the n real rows
+      float m = -INFINITY;
+      for (int r = lane; r < n; r += 32) m = fmaxf(m, xs[r]);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float s = 0.f;
+      for (int r = lane; r < n; r += 32) s += expf(xs[r] - m);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) stat[0] = m + logf(s);
+    }
+    __syncthreads();
+    lse = stat[0];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) { kt[k] = 0.f; vt[k] = 0.f; }
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int r = g + 16 * it;
+      const float w = (r < n) ? expf(x[it] - lse) : 0.f;
+      float fk[8], fv[8];
+      bf16x8_to_f32(kr[it], fk);
+      bf16x8_to_f32(vr[it], fv);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        kt[k] = fmaf(w, fk[k], kt[k]);
+        vt[k] = fmaf(w, fv[k], vt[k]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) vt[k] = 0.f;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      float fv[8];
+      bf16x8_to_f32(vr[it], fv);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) vt[k] += fv[k];
+    }
+  }
+
+  const float inv_n = 1.f / static_cast<float>(n);
+  const float ksum_d = cta_sum_over_rows(ks, red, c);
+  const float vt_d = cta_sum_over_rows(vt, red, c);
+  float kt_d = 0.f;
+  if (kVariant == 0) kt_d = cta_sum_over_rows(kt, red, c);
+
+  const size_t o = (bh * nb + blk) * kDim + tid;
+  if (tid < kDim) kpool[o] = ksum_d * inv_n;
+  if (kVariant == 0) {
+    // bias = LSE - anchor . bf16(k~) * scale  (bf16(k~) is what the MMA sees)
+    const float kt_b = bf16_round(kt_d);
+    float p = (tid < kDim) ? __ldg(anchor + bh * kDim + tid) * kt_b : 0.f;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+    if (lane == 0 && warp < 4) red[warp] = p;
+    __syncthreads();
+    if (tid < kDim) {
+      ksum[o] = __float2bfloat16_rn(kt_d);
+      vsum[o] = __float2bfloat16_rn(vt_d);
+    }
+    if (tid == 0) bias[bh * nb + blk] = lse - ((red[0] + red[1]) + (red[2] + red[3])) * scale;
+  } else {
+    if (tid < kDim) {
+      ksum[o] = __float2bfloat16_rn(ksum_d * inv_n);
+      vsum[o] = __float2bfloat16_rn(vt_d * inv_n);
+    }
+    if (tid == 0) bias[bh * nb + blk] = logf(static_cast<float>(n));
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Shape& s, const void* Q, float* qpool, float* anchor,
+                        cudaStream_t st) {
+  const dim3 grid(s.nb, s.B * s.H);
+  pool_q_kernel<<<grid, kThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(Q), qpool, s.N,
+                                           s.nb);
+  anchor_kernel<<<s.B * s.H, 1024, 0, st>>>(qpool, anchor, s.N, s.nb, s.pb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const float* anchor,
+                             float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st) {
+  const dim3 grid(s.nb, s.B * s.H);
+  const float scale = 0.088388347648318440550f;  // 1 / sqrt(128)
+  auto Kp = static_cast<const __nv_bfloat16*>(K);
+  auto Vp = static_cast<const __nv_bfloat16*>(V);
+  auto ks = static_cast<__nv_bfloat16*>(ksum);
+  auto vs = static_cast<__nv_bfloat16*>(vsum);
+  if (s.variant == 0)
+    summarize_kernel<0><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias, s.N, s.nb,
+                                                   scale);
+  else
+    summarize_kernel<1><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias, s.N, s.nb,
+                                                   scale);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

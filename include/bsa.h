@@ -1,0 +1,165 @@
+/*
+ * bsa.h -- C ABI of libbsa.so: block-sparse video self-attention forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (sources are web pages, cited by title and section):
+ *   "h3-sparse-attn 0.1.0" (PyPI project page), opening description: each
+ *   query block of 128 tokens attends to its top-k key blocks; the skipped
+ *   key blocks are folded back in as one summary row each.  Section "Use":
+ *   top_k counts 128-token key blocks.
+ *   "Spark-H3: Block Sparse Attention Speeds Up MiniMax-H3 in ComfyUI",
+ *   section "What Spark-Attn changes": exact branch + compressed branch; the
+ *   Spark-Reweight bullet: weighted summaries plus a log-mass bias, with the
+ *   mean of the video queries as one anchor per head.
+ *   "H3 Sparse Attention" (comfy.icu WAS node and video_budget node): prompt /
+ *   text rows are read exactly and stay dense (the optional dense prefix).
+ *
+ * Conventions shared by every entry point
+ *   - Q, K, V, O are bf16 [B, H, N, D] contiguous (row-major, D fastest),
+ *     D == 128.  Their base addresses must be 16-byte aligned (the kernels
+ *     stage them with TMA), otherwise BSA_ERR_ALIGN.
+ *   - Block size 128; nb = ceil(N / 128); the last block may be ragged.
+ *     pb = prefix / 128 dense-prefix blocks, nbv = nb - pb video blocks,
+ *     k_eff = min(top_k, nbv).
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, except
+ *     in bsa_forward_host, whose h* arguments are HOST pointers.  The library
+ *     allocates no memory and keeps no per-call state.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on that stream: a return of BSA_OK
+ *     means the arguments were valid and the kernels were enqueued without a
+ *     launch error; device-side completion is observed by synchronising.
+ *   - On any error nothing is enqueued (argument checks run before the first
+ *     launch) except BSA_ERR_CUDA, which reports cudaGetLastError() after a
+ *     launch.
+ *   - The library is thread-safe for concurrent calls on different streams;
+ *     calls on one stream are ordered by that stream.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID = 1,     /* bad size, range, variant or null pointer   */
+  BSA_ERR_ALIGN = 2,       /* a pointer is not 16-byte aligned           */
+  BSA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed       */
+  BSA_ERR_TIMEOUT = 4,     /* written to *dev_status by a kernel whose
+                              bounded wait expired (never returned)      */
+  BSA_ERR_UNSUPPORTED = 5  /* device is not sm_100 / driver lacks TMA    */
+} bsa_status;
+
+typedef enum {
+  BSA_SUMMARY_ANCHOR = 0,  /* Spark-Reweight: softmax-at-the-anchor weighted
+                              k~, v~; bias = ln n + (LSE - ln n - qbar.k~/sqrt d) */
+  BSA_SUMMARY_MEAN = 1     /* mean-pooled k~, v~; bias = ln n            */
+} bsa_variant;
+
+typedef struct {
+  int32_t B, H, N, D;   /* D must be 128; B, H >= 1; 1 <= N <= 2^21          */
+  int32_t top_k;        /* >= 1; clamped to nbv                              */
+  int32_t prefix;       /* dense-prefix tokens: multiple of 128, 0 <= prefix < N */
+  int32_t variant;      /* bsa_variant                                       */
+  int32_t* dev_status;  /* optional device int (may be NULL).  Kernels with
+                           bounded waits write BSA_ERR_TIMEOUT there if a wait
+                           expires (~2 s); the caller zeroes it beforehand.  */
+} bsa_params;
+
+/* ---- sizes ------------------------------------------------------------ */
+
+/* nb = ceil(N / 128), or -1 if p is invalid. */
+int32_t bsa_num_blocks(const bsa_params* p);
+
+/* kcap: row length of the idx array written by bsa_select,
+ * = nb if prefix > 0 (prefix query rows list every block), else pb + k_eff.
+ * Returns -1 if p is invalid. */
+int32_t bsa_select_capacity(const bsa_params* p);
+
+/* Bytes of the workspace bsa_forward / bsa_forward_host need (256-byte
+ * aligned sub-buffers: qpool, anchor, kpool, ksum, vsum, bias, idx, cnt).
+ * Returns 0 if p is invalid. */
+size_t bsa_workspace_bytes(const bsa_params* p);
+
+/* ---- the four stages -------------------------------------------------- */
+
+/* Step 1-2 (pool + anchor).  Per (b, h): qpool[i] = mean of the real query
+ * rows of block i (fp32 [B,H,nb,D]); anchor = mean of the video query rows
+ * t >= prefix (fp32 [B,H,D]) -- "the mean of the video queries as one anchor
+ * per head" (Spark-H3 page, Spark-Reweight bullet).  Reads Q once.
+ * Deterministic (fixed reduction order). */
+int bsa_pool(const bsa_params* p, const void* Q, float* qpool, float* anchor,
+             void* stream);
+
+/* Step 1 + 3 (key pooling and one summary row per key block), fused so K and
+ * V are each read once.  Outputs, all [B,H,nb,...]:
+ *   kpool fp32 [.., D]  mean of the real keys of block j;
+ *   ksum  bf16 [.., D]  k~_j;   vsum bf16 [.., D]  v~_j;   bias fp32 [..]  bias_j.
+ * ANCHOR variant: x_t = anchor . k_t / sqrt(D), w = softmax_t(x) over the
+ * block, k~ = sum w k, v~ = sum w v, bias = LSE(x) - anchor . bf16(k~) / sqrt(D)
+ * (the ln n_j terms of ln n + (LSE - ln n - ..) cancel; bf16(k~) is the value
+ * the attention MMA later uses).  MEAN variant: k~ = mean k, v~ = mean v,
+ * bias = ln n_j; `anchor` may then be NULL.  Summaries of prefix blocks are
+ * computed but never used. */
+int bsa_summarize(const bsa_params* p, const void* K, const void* V,
+                  const float* anchor, float* kpool, void* ksum, void* vsum,
+                  float* bias, void* stream);
+
+/* Step 4-5 (block score + top-k).  S_ij = qpool_i . kpool_j / sqrt(D) in fp32
+ * for video key blocks j >= pb.  Video query block i >= pb keeps the k_eff
+ * largest S_ij, ties to the lower j, and writes
+ *   idx[b,h,i,:] = 0..pb-1 followed by the chosen j ascending, then -1 padding
+ *   (int32 [B,H,nb,kcap]),  cnt[b,h,i] = pb + k_eff  (int32 [B,H,nb]).
+ * Prefix query block i < pb lists every block: idx = 0..nb-1, cnt = nb.
+ * Deterministic. */
+int bsa_select(const bsa_params* p, const float* qpool, const float* kpool,
+               int32_t* idx, int32_t* cnt, void* stream);
+
+/* Step 6 (exact branch + compressed branch + epilogue).  For query row t of
+ * block i: logits q_t.k_u/sqrt(D) for the tokens u of the blocks idx[b,h,i,
+ * 0..cnt) (ragged tail masked) and, for a video query block, q_t.k~_j/sqrt(D)
+ * + bias_j for every video block j not listed; O_t = softmax(logits) @ [V ; v~]
+ * written as bf16.  lse (fp32 [B,H,N], natural log) is written when non-NULL.
+ * tcgen05 MMA (bf16 in, fp32 accumulate in TMEM), online softmax in fp32.
+ * idx/cnt must be what bsa_select wrote for the same parameters. */
+int bsa_attend(const bsa_params* p, const void* Q, const void* K, const void* V,
+               const int32_t* idx, const int32_t* cnt, const void* ksum,
+               const void* vsum, const float* bias, void* O, float* lse,
+               void* stream);
+
+/* ---- whole path ------------------------------------------------------- */
+
+/* bsa_pool, bsa_summarize, bsa_select, bsa_attend in order on `stream`.
+ * `workspace` is a caller-owned device buffer of at least
+ * bsa_workspace_bytes(p) bytes, 256-byte aligned. */
+int bsa_forward(const bsa_params* p, const void* Q, const void* K, const void* V,
+                void* O, float* lse, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/* bsa_forward from HOST buffers: copies hQ, hK, hV (bf16 [B,H,N,D], pinned
+ * for asynchronous copies) to the caller's device buffers dQ, dK, dV with one
+ * cudaMemcpyAsync each, runs bsa_forward, and copies dO back to hO (and dlse
+ * to hlse when both are non-NULL), all on `stream`.  Returns after enqueueing;
+ * synchronise the stream before reading hO. */
+int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK,
+                     const void* hV, void* hO, float* hlse, void* dQ, void* dK,
+                     void* dV, void* dO, float* dlse, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* Human-readable name of a bsa_status value (static string). */
+const char* bsa_status_string(int status);
+
+/* Launches a single-CTA kernel that waits on a barrier nothing will ever
+ * release, bounded by timeout_ns, then writes BSA_ERR_TIMEOUT to *dev_status
+ * and returns.  Exists so tests can check on a GPU that an expired wait ends
+ * with a status the host can read and leaves the context usable. */
+int bsa_debug_expired_wait(int32_t* dev_status, uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H_ */

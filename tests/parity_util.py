@@ -1,0 +1,131 @@
+"""Comparison helpers for the GPU-vs-oracle parity tests (acceptance rules of
+the spec: indices exact except at score gaps under 1e-5; O max-abs <= 2e-2 and
+rel-L2 <= 1e-2 against the fp64 oracle)."""
+
+import numpy as np
+import torch
+
+import oracle as orc
+from block_sparse_video_bsa_b200 import bsa
+
+TIE_GAP = 1e-5
+O_MAX_ABS = 2e-2
+O_REL_L2 = 1e-2
+POOL_RTOL, POOL_ATOL = 1e-5, 1e-6
+SUM_RTOL, SUM_ATOL = 2.0 ** -7, 1e-3
+# bf16 unit roundoff.  The GPU feeds bf16(k~) to the MMA and computes its
+# bias from the same bf16(k~), so (exactly, up to fp32 slack)
+#   z_gpu(q) - z_ref(q) = (q - qbar) . (bf16(k~) - k~) / sqrt(d),
+# bounded by 2^-8 * sum_d |q_d - qbar_d| |k~_d| / sqrt(d); the bias alone moves
+# by the same expression at q = 0.  (Mean variant: bias = ln n has no k~
+# term and the logit shift is q . (bf16(k~) - k~) / sqrt(d).)  lse moves by at
+# most the largest shift of any summary logit.  These bounds use oracle values
+# only.
+BF16_U = 2.0 ** -8
+FP32_SLACK = 2e-4
+
+
+def run_stages(Q, K, V, top_k, prefix, variant, with_lse=True):
+    """Every stage through its own C entry point; returns all device outputs."""
+    B, H, N, _ = Q.shape
+    p = bsa.params(B, H, N, top_k, prefix, variant)
+    buf = bsa.stage_buffers(B, H, N, top_k, prefix, variant, device=Q.device)
+    bsa.bsa_pool(p, Q, buf["qpool"], buf["anchor"])
+    bsa.bsa_summarize(p, K, V, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"], buf["bias"])
+    bsa.bsa_select(p, buf["qpool"], buf["kpool"], buf["idx"], buf["cnt"])
+    O = torch.empty_like(Q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=Q.device) if with_lse else None
+    bsa.bsa_attend(p, Q, K, V, buf["idx"], buf["cnt"], buf["ksum"], buf["vsum"], buf["bias"],
+                   O, lse)
+    torch.cuda.synchronize()
+    buf["O"] = O
+    buf["lse"] = lse
+    return buf
+
+
+def host(t):
+    return t.detach().float().cpu().double().numpy() if t.dtype == torch.bfloat16 \
+        else t.detach().cpu().numpy()
+
+
+def check_selection(idx_row_block, cnt_row, ref, prefix_blocks, top_k):
+    """idx/cnt of one head vs the oracle's lists; returns query blocks with a
+    near-tie swap (allowed only where the oracle's scores are within 1e-5 of
+    the k-th score)."""
+    S, lists = ref["scores"], ref["lists"]
+    nb = S.shape[0]
+    pb = prefix_blocks
+    k_eff = min(top_k, nb - pb)
+    swapped = set()
+    for i in range(nb):
+        want = list(lists[i])
+        c = int(cnt_row[i])
+        assert c == len(want), (i, c, len(want))
+        got = [int(v) for v in idx_row_block[i, :c]]
+        assert all(int(v) == -1 for v in idx_row_block[i, c:]), f"padding of row {i}"
+        if got == want:
+            continue
+        assert i >= pb, f"prefix row {i} differs"
+        assert got[:pb] == list(range(pb))
+        assert got == sorted(set(got)) and all(pb <= j < nb for j in got[pb:])
+        cand = np.arange(pb, nb)
+        kth = np.sort(S[i, cand])[::-1][k_eff - 1]
+        for j in set(got) ^ set(want):
+            assert abs(S[i, j] - kth) < TIE_GAP, (i, j, S[i, j], kth)
+        swapped.add(i)
+    return swapped
+
+
+def rows_of_blocks(N, blocks):
+    rows = []
+    for i in sorted(blocks):
+        a, b = orc.block_bounds(N)[i]
+        rows.extend(range(a, b))
+    return np.array(rows, dtype=np.int64)
+
+
+def check_output(O_gpu, O_ref, N, exclude_blocks=()):
+    keep = np.ones(N, dtype=bool)
+    if exclude_blocks:
+        keep[rows_of_blocks(N, exclude_blocks)] = False
+    g, r = O_gpu[keep], O_ref[keep]
+    err = np.abs(g - r)
+    max_abs = float(err.max()) if err.size else 0.0
+    rel_l2 = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30))
+    assert max_abs <= O_MAX_ABS, f"max-abs {max_abs}"
+    assert rel_l2 <= O_REL_L2, f"rel-L2 {rel_l2}"
+    return max_abs, rel_l2
+
+
+def check_head(buf, Q, K, V, b, h, top_k, prefix, variant, check_lse=True):
+    """Full per-stage parity of one (b, h) slice; returns (max_abs, rel_l2, swaps)."""
+    N = Q.shape[2]
+    ref = orc.forward_head(host(Q[b, h]), host(K[b, h]), host(V[b, h]), top_k, prefix, variant)
+    pb = prefix // 128
+    np.testing.assert_allclose(host(buf["qpool"][b, h]), ref["qpool"], rtol=POOL_RTOL, atol=POOL_ATOL)
+    np.testing.assert_allclose(host(buf["kpool"][b, h]), ref["kpool"], rtol=POOL_RTOL, atol=POOL_ATOL)
+    np.testing.assert_allclose(host(buf["anchor"][b, h]), ref["anchor"], rtol=POOL_RTOL,
+                               atol=POOL_ATOL)
+    v = slice(pb, None)  # summaries of prefix blocks are never used
+    np.testing.assert_allclose(host(buf["ksum"][b, h])[v], ref["ksum"][v], rtol=SUM_RTOL, atol=SUM_ATOL)
+    np.testing.assert_allclose(host(buf["vsum"][b, h])[v], ref["vsum"][v], rtol=SUM_RTOL, atol=SUM_ATOL)
+    d = ref["ksum"].shape[1]
+    kabs = np.abs(ref["ksum"][v])
+    bias_tol = BF16_U * (kabs @ np.abs(ref["anchor"])) / np.sqrt(d) + FP32_SLACK
+    bias_err = np.abs(host(buf["bias"][b, h])[v] - ref["bias"][v])
+    assert (bias_err <= bias_tol).all(), f"bias err {bias_err.max()} > {bias_tol.min()}"
+    swaps = check_selection(host(buf["idx"][b, h]), host(buf["cnt"][b, h]), ref, pb, top_k)
+    m, r = check_output(host(buf["O"][b, h]), ref["O"], N, swaps)
+    if check_lse and buf.get("lse") is not None:
+        keep = np.ones(N, dtype=bool)
+        if swaps:
+            keep[rows_of_blocks(N, swaps)] = False
+        # anchor variant: the shift is (q - qbar) . delta; mean variant: q . delta
+        centre = ref["anchor"][None, :] if variant == "anchor" else 0.0
+        qd = np.abs(host(Q[b, h]) - centre)
+        lse_tol = BF16_U * (qd @ kabs.T).max(axis=1) / np.sqrt(d) + FP32_SLACK \
+            if kabs.size else np.full(N, FP32_SLACK)
+        lse_err = np.abs(host(buf["lse"][b, h]) - ref["lse"])
+        assert (lse_err[keep] <= lse_tol[keep]).all(), \
+            f"lse err {lse_err[keep].max()} (bound {lse_tol[keep].min()})"
+    return m, r, swaps

@@ -1,0 +1,89 @@
+"""The C ABI without a GPU: libbsa.so loads, exports every function that
+include/bsa.h declares, and the host-side checks (sizes, bad arguments) that
+run before any CUDA call behave as documented.  No compute call here touches
+the device: every call below returns from argument validation."""
+
+import ctypes
+
+import pytest
+
+from block_sparse_video_bsa_b200 import bsa
+
+
+@pytest.fixture(scope="module")
+def L():
+    return bsa.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = bsa.header_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(bsa._SIGS), "binding and header disagree"
+
+
+def _p(**kw):
+    base = dict(B=1, H=56, N=37_740, top_k=64, prefix=0, variant="anchor")
+    base.update(kw)
+    return bsa.params(**base)
+
+
+def test_sizes_match_the_block_arithmetic():
+    p = _p()
+    assert bsa.bsa_num_blocks(p) == 295
+    assert bsa.bsa_select_capacity(p) == 64
+    assert bsa.bsa_select_capacity(_p(N=103_996, prefix=512)) == 813
+    assert bsa.bsa_select_capacity(_p(top_k=1000)) == 295       # clamped to nbv
+    assert bsa.bsa_num_blocks(_p(N=1)) == 1
+    ws = bsa.bsa_workspace_bytes(p)
+    blocks = 56 * 295
+    want = blocks * 128 * 4 * 2 + 56 * 128 * 4 + blocks * 128 * 2 * 2 + blocks * 4 \
+        + blocks * 64 * 4 + blocks * 4
+    assert want <= ws <= want + 8 * 256
+
+
+@pytest.mark.parametrize("kw", [dict(D=64), dict(top_k=0), dict(prefix=100), dict(prefix=37_760),
+                                dict(N=0), dict(B=0), dict(variant=7), dict(N=(1 << 21) + 1),
+                                dict(H=70_000)])
+def test_invalid_parameters_rejected_before_launch(kw):
+    p = _p(**kw)
+    assert bsa.bsa_num_blocks(p) == -1
+    assert bsa.bsa_workspace_bytes(p) == 0
+    rc = bsa.lib().bsa_pool(ctypes.byref(p), ctypes.c_void_p(4096), ctypes.c_void_p(4096),
+                            ctypes.c_void_p(4096), None)
+    assert rc == bsa.BSA_ERR_INVALID
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch():
+    L = bsa.lib()
+    p = _p()
+    P = ctypes.byref(p)
+    a = ctypes.c_void_p(1 << 20)       # never dereferenced: validation fails first
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert L.bsa_pool(P, None, a, a, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_pool(P, odd, a, a, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_summarize(P, a, a, None, a, a, a, a, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_select(P, a, a, None, a, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_attend(P, a, a, a, a, a, a, a, a, None, None, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_attend(P, a, a, a, a, a, a, a, a, odd, None, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_forward(P, a, a, a, a, None, a, 16, None) == bsa.BSA_ERR_INVALID  # too small
+    assert L.bsa_forward(P, a, a, a, a, None, odd, 1 << 40, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_forward_host(P, a, a, a, a, None, a, a, a, None, None, a, 1 << 40,
+                              None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_debug_expired_wait(None, 1000, None) == bsa.BSA_ERR_INVALID
+    # the mean variant does not need an anchor; the anchor variant does
+    pm = _p(variant="mean")
+    assert L.bsa_summarize(ctypes.byref(pm), a, a, None, a, a, a, a, None) != bsa.BSA_ERR_INVALID
+
+
+def test_status_strings():
+    assert bsa.status_string(bsa.BSA_OK) == "ok"
+    assert "aligned" in bsa.status_string(bsa.BSA_ERR_ALIGN)
+    assert bsa.status_string(99) == "unknown status"
+
+
+def test_density_to_topk_rounds_up():
+    assert [bsa.topk_from_density(r, 133_644) for r in (0.1, 0.2, 0.3)] == [105, 209, 314]
+    assert bsa.topk_from_density(0.3, 128_000) == 300
+    assert bsa.topk_from_density(0.001, 2048) == 1

@@ -1,0 +1,169 @@
+"""GPU parity: every stage of the CUDA path (through the C ABI) against the
+fp64 oracle on the same seeded bf16 inputs.  Small cases are compared in
+full; the five workloads at full size are compared on seeded head samples,
+in the launch configuration bench.py times."""
+
+import random
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from block_sparse_video_bsa_b200 import bsa
+from block_sparse_video_bsa_b200.inputs import CONFIGS, make_qkv
+
+from parity_util import check_head, check_output, host, run_stages
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(B, H, N, kind, seed=0):
+    return make_qkv(B, H, N, 128, kind, seed, device="cuda")
+
+
+@pytest.mark.parametrize("B,H,N,top_k,prefix,variant,kind", [
+    (1, 2, 2048, 4, 0, "mean", "iid"),                 # the small iid workload
+    (1, 2, 2048, 4, 0, "anchor", "iid"),
+    (2, 2, 1000, 3, 0, "anchor", "block_offset"),      # ragged tail (104 rows)
+    (1, 3, 1500, 2, 256, "anchor", "block_offset"),    # dense prefix + ragged (92)
+    (1, 2, 1500, 2, 256, "mean", "block_offset"),
+    (1, 2, 4100, 5, 0, "anchor", "block_offset"),      # ragged tail of 4 rows, 33 blocks
+    (1, 1, 300, 1, 0, "anchor", "iid"),                # 3 blocks, k=1
+    (1, 2, 2000, 15, 0, "anchor", "block_offset"),     # k_eff = nbv - 1: one summary
+    (1, 1, 17_000, 7, 0, "anchor", "block_offset"),    # 133 blocks: 2 summary tiles
+])
+def test_small_cases_all_stages(B, H, N, top_k, prefix, variant, kind):
+    Q, K, V = _inputs(B, H, N, kind)
+    buf = run_stages(Q, K, V, top_k, prefix, variant)
+    for b in range(B):
+        for h in range(H):
+            check_head(buf, Q, K, V, b, h, top_k, prefix, variant)
+
+
+@pytest.mark.parametrize("N", [1, 100, 127, 128, 129, 255, 383])
+def test_edge_lengths(N):
+    # one block (possibly a single token), block boundaries, ragged tails
+    Q, K, V = _inputs(1, 2, N, "iid", seed=N)
+    for variant in ("anchor", "mean"):
+        buf = run_stages(Q, K, V, 1, 0, variant)
+        for h in range(2):
+            check_head(buf, Q, K, V, 0, h, 1, 0, variant)
+
+
+@pytest.mark.parametrize("N,prefix", [(1000, 0), (1500, 256), (1, 0)])
+def test_topk_all_blocks_equals_dense_sdpa(N, prefix):
+    Q, K, V = _inputs(1, 2, N, "block_offset", seed=3)
+    O = bsa.forward(Q, K, V, top_k=10_000, prefix=prefix)
+    torch.cuda.synchronize()
+    dense = torch.nn.functional.scaled_dot_product_attention(Q.float(), K.float(), V.float())
+    err = (O.float() - dense).abs().max().item()
+    assert err <= 2e-2
+    ref = orc.forward_head(host(Q[0, 0]), host(K[0, 0]), host(V[0, 0]), 10_000, prefix)["O"]
+    check_output(host(O[0, 0]), ref, N)
+
+
+def test_equal_scores_select_lowest_indices():
+    # every key block identical -> every score equal -> blocks pb..pb+k-1
+    N, pb = 2048, 2
+    Q, K, V = _inputs(1, 1, N, "iid", seed=5)
+    K[:] = K[:, :, :128].repeat(1, 1, N // 128, 1)
+    buf = run_stages(Q, K, V, 3, pb * 128, "anchor")
+    idx, cnt = host(buf["idx"][0, 0]), host(buf["cnt"][0, 0])
+    for i in range(pb, N // 128):
+        assert list(idx[i, :cnt[i]]) == [0, 1, 2, 3, 4]
+    check_head(buf, Q, K, V, 0, 0, 3, pb * 128, "anchor")
+
+
+def test_forward_matches_stages_and_is_deterministic():
+    N, top_k = 3000, 4
+    Q, K, V = _inputs(1, 4, N, "block_offset", seed=9)
+    buf = run_stages(Q, K, V, top_k, 0, "anchor")
+    O1, l1 = bsa.forward(Q, K, V, top_k, return_lse=True)
+    O2, l2 = bsa.forward(Q, K, V, top_k, return_lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, buf["O"]) and torch.equal(O1, O2)
+    assert torch.equal(l1, buf["lse"]) and torch.equal(l1, l2)
+
+
+def test_forward_host_buffers_match_device_path():
+    B, H, N, top_k = 1, 2, 2500, 3
+    Q, K, V = _inputs(B, H, N, "block_offset", seed=11)
+    p = bsa.params(B, H, N, top_k)
+    ws = bsa.workspace(p)
+    hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+    hO = torch.empty_like(hQ).pin_memory()
+    hl = torch.empty(B, H, N, dtype=torch.float32).pin_memory()
+    dQ, dK, dV, dO = (torch.empty_like(Q) for _ in range(4))
+    dl = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    bsa.bsa_forward_host(p, hQ, hK, hV, hO, hl, dQ, dK, dV, dO, dl, ws)
+    torch.cuda.synchronize()
+    O, lse = bsa.forward(Q, K, V, top_k, return_lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(hO, O.cpu()) and torch.equal(hl, lse.cpu())
+
+
+def test_expired_wait_reports_timeout_and_context_survives():
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bsa.bsa_debug_expired_wait(status, 50_000_000)   # 50 ms, nothing will arrive
+    torch.cuda.synchronize()
+    assert int(status.item()) == bsa.BSA_ERR_TIMEOUT
+    Q, K, V = _inputs(1, 1, 512, "iid")
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    p = bsa.params(1, 1, 512, 2, dev_status=st2)
+    O = torch.empty_like(Q)
+    bsa.bsa_forward(p, Q, K, V, O, None, bsa.workspace(p))
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 0
+    assert torch.isfinite(O.float()).all()
+
+
+def test_device_errors_are_reported_not_hidden():
+    Q, K, V = _inputs(1, 1, 256, "iid")
+    p = bsa.params(1, 1, 256, 1)
+    O = torch.empty_like(Q)
+    with pytest.raises(bsa.BsaError):
+        bsa.bsa_forward(p, Q, K, V, O, None, torch.empty(16, dtype=torch.uint8, device="cuda"))
+
+
+def _sample_heads(H, n, seed=0):
+    return sorted(random.Random(seed).sample(range(H), n))
+
+
+@pytest.mark.parametrize("name,n_heads", [("h3_768p_5s", 2), ("h3_768p_10s", 1),
+                                          ("h3_768p_15s_prefix512", 1), ("h3_2k_5s", 1)])
+def test_full_size_workloads_on_sampled_heads(name, n_heads):
+    cfg = CONFIGS[name]
+    B, H, N = cfg["B"], cfg["H"], cfg["N"]
+    Q, K, V = _inputs(B, H, N, cfg["kind"])
+    p = bsa.params(B, H, N, cfg["top_k"], cfg["prefix"], cfg["variant"])
+    O = torch.empty_like(Q)
+    bsa.bsa_forward(p, Q, K, V, O, None, bsa.workspace(p))       # the benchmarked call
+    buf = run_stages(Q, K, V, cfg["top_k"], cfg["prefix"], cfg["variant"], with_lse=False)
+    assert torch.equal(O, buf["O"])
+    for h in _sample_heads(H, n_heads, seed=len(name)):
+        m, r, swaps = check_head(buf, Q, K, V, 0, h, cfg["top_k"], cfg["prefix"], cfg["variant"],
+                                 check_lse=False)
+        assert len(swaps) <= 2
+    del Q, K, V, O, buf
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("top_k", [16, 128])
+def test_topk_sweep_sampled_head(top_k):
+    cfg = CONFIGS["h3_768p_10s"]
+    B, H, N = 1, 4, cfg["N"]     # 4 heads of the sweep workload, one checked
+    Q, K, V = _inputs(B, H, N, cfg["kind"])
+    buf = run_stages(Q, K, V, top_k, 0, "anchor", with_lse=False)
+    check_head(buf, Q, K, V, 0, 2, top_k, 0, "anchor", check_lse=False)
+
+
+@pytest.mark.parametrize("rho", [0.3])
+def test_density_sweep_sampled_head(rho):
+    cfg = CONFIGS["h3_2k_5s"]
+    N = cfg["N"]
+    top_k = bsa.topk_from_density(rho, N)
+    assert top_k == 314
+    Q, K, V = _inputs(1, 2, N, cfg["kind"])
+    buf = run_stages(Q, K, V, top_k, 0, "anchor", with_lse=False)
+    check_head(buf, Q, K, V, 0, 1, top_k, 0, "anchor", check_lse=False)
