@@ -19,7 +19,9 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbsa.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "bsa.h")
 
-BSA_OK, BSA_ERR_INVALID, BSA_ERR_ALIGN, BSA_ERR_CUDA, BSA_ERR_TIMEOUT, BSA_ERR_UNSUPPORTED = range(6)
+(BSA_OK, BSA_ERR_INVALID, BSA_ERR_ALIGN, BSA_ERR_CUDA, BSA_ERR_TIMEOUT, BSA_ERR_UNSUPPORTED,
+ BSA_ERR_SCRATCH) = range(7)
+BSA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 VARIANTS = {"anchor": 0, "mean": 1}
 
 
@@ -53,6 +55,7 @@ _SIGS = {
                                         _vp, ctypes.c_size_t, _vp]),
     "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_debug_expired_wait": (ctypes.c_int, [_vp, ctypes.c_uint64, _vp]),
+    "bsa_forward_noalloc": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 
 
@@ -152,6 +155,13 @@ def bsa_forward_host(p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, s
                                   _ptr(hlse), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dO), _ptr(dlse),
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream)), "bsa_forward_host")
+
+
+def bsa_forward_noalloc(p, Q, K, V, O, lse=None, stream=None):
+    """bsa_forward with its workspace in the library's static device scratch,
+    for callers that cannot allocate device memory (see include/bsa.h)."""
+    _check(lib().bsa_forward_noalloc(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                     _ptr(lse), _stream(stream)), "bsa_forward_noalloc")
 
 
 def bsa_debug_expired_wait(dev_status, timeout_ns: int, stream=None):

@@ -285,6 +285,7 @@ const char* bsa_status_string(int status) {
     case BSA_ERR_CUDA: return "CUDA error";
     case BSA_ERR_TIMEOUT: return "bounded device wait expired";
     case BSA_ERR_UNSUPPORTED: return "unsupported device (needs sm_100) or driver";
+    case BSA_ERR_SCRATCH: return "problem exceeds the static scratch of bsa_forward_noalloc";
     default: return "unknown status";
   }
 }

@@ -51,7 +51,9 @@ typedef enum {
   BSA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed       */
   BSA_ERR_TIMEOUT = 4,     /* written to *dev_status by a kernel whose
                               bounded wait expired (never returned)      */
-  BSA_ERR_UNSUPPORTED = 5  /* device is not sm_100 / driver lacks TMA    */
+  BSA_ERR_UNSUPPORTED = 5, /* device is not sm_100 / driver lacks TMA    */
+  BSA_ERR_SCRATCH = 6      /* bsa_forward_noalloc: the problem needs more
+                              workspace than its static scratch holds    */
 } bsa_status;
 
 typedef enum {
@@ -149,6 +151,37 @@ int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK,
                      const void* hV, void* hO, float* hlse, void* dQ, void* dK,
                      void* dV, void* dO, float* dlse, void* workspace,
                      size_t workspace_bytes, void* stream);
+
+/* ---- forward without any allocation ---------------------------------- */
+
+/* Size of the static device scratch behind bsa_forward_noalloc: 64 MiB. */
+#define BSA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* bsa_forward for callers that cannot allocate device memory.  The pages
+ * describe nothing like it (it has no counterpart there); it exists for hosts
+ * where cudaMalloc is not an option: a plugin inside a framework whose memory
+ * pool owns the device, a server that reserves all memory at start-up and
+ * treats later allocations as faults, or latency-critical code that cannot
+ * take cudaMalloc's implicit device synchronisation.
+ *
+ * Same arguments and results as bsa_forward, minus the workspace: the
+ * intermediates live in a file-scope static device array of
+ * BSA_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
+ * until the process exits.  The call allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine); the caller still passes Q, K, V,
+ * O and the optional lse.
+ *   - Problems whose bsa_workspace_bytes(p) exceeds the scratch size are
+ *     rejected with BSA_ERR_SCRATCH before anything is enqueued (64 MiB covers
+ *     e.g. B=1, H=56, N=73,416, top_k=64).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array per device and it keeps the last call's
+ *     contents.  No part of it needs to start at zero (every stage fully
+ *     writes what the next stage reads), but calls that overlap on the GPU
+ *     (e.g. on two streams without ordering) race on it: order them. */
+int bsa_forward_noalloc(const bsa_params* p, const void* Q, const void* K, const void* V,
+                        void* O, float* lse, void* stream);
 
 /* Human-readable name of a bsa_status value (static string). */
 const char* bsa_status_string(int status);
