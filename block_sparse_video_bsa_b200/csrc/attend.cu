@@ -1,34 +1,40 @@
 // Exact branch + compressed branch of block-sparse attention on tcgen05.
 //
-// "Block sparse attention splits a video attention pass into two branches:
-// an exact branch that computes the top-ranked key/value blocks in full, and
-// a compressed branch that covers everything else" (Spark-H3 page, section
-// "What Spark-Attn changes").  For one query block (128 rows) this kernel
-// streams, as 128-key tiles:
+// Spark-H3 page, section "What Spark-Attn changes": attention is split into
+// an exact branch, which computes the highest-ranked key/value blocks in
+// full, and a cheap compressed branch for all other blocks.  For one query
+// block (128 rows) this kernel streams 128-key tiles:
 //   * the listed key blocks idx[0..cnt) (exact branch; the ragged last block
 //     is masked by column), then
-//   * the summary rows k~_j / v~_j of all video blocks, 128 per tile, with
-//     logit + bias_j, and the listed / prefix / out-of-range columns masked
+//   * the summary rows k~_j / v~_j of the video blocks, 128 per tile, with
+//     logit + bias_j and the listed / prefix / out-of-range columns masked
 //     (compressed branch),
 // through one online softmax, so both branches share the running max and sum.
 //
-// One CTA per query block, 256 threads in four roles:
-//   warp 0      TMA producer: Q once, then K / V tiles gathered by block index
-//               (3-D tensor maps [B*H, rows, 128], 128-byte swizzle; rows past
-//               the end of a head are zero-filled by the TMA unit).
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer:
-//               S[t&1] = Q K_t^T  (M=N=128, K=128, both K-major), then
-//               O     += P_t V_t  (A = P from shared memory, B = V MN-major).
-//   warps 4-7   softmax: one thread per query row (TMEM lane = row), fp32
-//               online softmax in base 2 with lazy rescaling of O (only when
-//               the running max grows by more than 2^8), P written as bf16
-//               into the swizzled shared-memory operand layout; epilogue
-//               O / l -> bf16 and lse.
-// TMEM: S0 cols [0,128), S1 [128,256), O [256,384) of a 512-column block.
-// Shared memory: Q 32 KB, K 2 x 32 KB, V 2 x 32 KB, P 32 KB, barriers, and a
-// bitmap of the listed blocks for masking the summary columns.
-// Every mbarrier wait is bounded (bsa_device.cuh); on expiry the CTA records
-// BSA_ERR_TIMEOUT, drains what it issued, frees TMEM and returns.
+// Each CTA runs TWO query blocks ("slots") of the same tile count side by
+// side, so the tensor core works on one slot while the other slot's softmax
+// runs.  384 threads in three warpgroups; the two softmax warpgroups raise
+// their register budget to 232 and the third lowers its own to 40
+// (128*40 + 256*232 = 384*168, the launch allocation):
+//   warps 0-3   softmax of slot 0, one thread per query row (TMEM lanes 0-127)
+//   warps 4-7   softmax of slot 1
+//   warp 8      TMA producer: Q0, Q1, then every K / V tile of both slots in
+//               exactly the order the MMA consumes them, through one ring of
+//               kRing 32 KB stages (3-D tensor maps [B*H, rows, 128], 128-byte
+//               swizzle; rows past the end of a head read as zero).
+//   warp 9      TMEM allocator + single-thread tcgen05.mma issuer:
+//                 S_s  = Q_s K^T          (A, B from shared memory, K-major)
+//                 O_s += P_s V            (A = P from TMEM, B = V MN-major)
+//               issue order S0(0) S1(0) | PV0(t) S0(t+1) PV1(t) S1(t+1) | ...
+//               MMAs of one thread execute in order, so S_s(t+1) overwrites
+//               the TMEM columns of P_s(t) only after PV_s(t) has read them.
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512);
+// P_s (bf16, two per 32-bit column) overlays the first 64 columns of S_s.
+// Softmax: fp32, base 2 (ex2.approx), lazy O rescale (only when the running
+// max grows by more than 2^8), P written with tcgen05.st; epilogue O / l ->
+// bf16 and lse.  Every mbarrier wait is bounded (bsa_device.cuh); on expiry
+// the CTA records BSA_ERR_TIMEOUT, drains what it issued, frees TMEM and
+// returns.
 #include "bsa_device.cuh"
 #include "bsa_kernels.h"
 
@@ -36,14 +42,16 @@ namespace bsa {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
+constexpr uint32_t kSoftmaxRegs = 232, kControlRegs = 40;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kRing = 5;
 constexpr uint32_t kTileBytes = 32768;   // 128 x 128 bf16
 constexpr uint32_t kSubBytes = 16384;    // 128 rows x 64 bf16 (one 128-byte swizzle atom wide)
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTileBytes;       // 2 stages
-constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;   // 2 stages
-constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;
-constexpr uint32_t kOffCtl = kOffP + kTileBytes;     // 196608
+constexpr uint32_t kOffQ = 0;            // Q0, Q1
+constexpr uint32_t kOffRing = 2 * kTileBytes;
+constexpr uint32_t kOffCtl = kOffRing + kRing * kTileBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr float kLog2e = 1.4426950408889634074f;
@@ -52,26 +60,26 @@ constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct Ctl {
-  uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, fin;
-  uint64_t bias_full[2];
+  uint64_t full[kRing], empty[kRing];
+  uint64_t q_full[2];
+  uint64_t s_full[2], p_full[2], o_final[2];
+  uint64_t bias_full[2][2];
+  uint64_t fin;
   uint32_t tmem_base;
   int abort_flag;
   int skip;
-  alignas(16) float bias_stage[2][128];   // masked bias of the current summary tile
-  uint32_t bitmap[1];   // ceil(nb / 32) words follow
+  alignas(16) float bias_stage[2][2][128];   // [slot][buffer][column]
 };
+static_assert(kOffCtl + sizeof(Ctl) <= 227 * 1024, "shared memory budget");
 
 struct Args {
   const int32_t* idx;
-  const int32_t* cnt;
   const float* bias;
   __nv_bfloat16* O;
   float* lse;
   int* dev_status;
   int N, nb, pb, nbv, k_eff, kcap, BH;
+  int prefix_ctas;    // CTAs that take dense-prefix query-block pairs
   float scale_log2;   // log2(e) / sqrt(128)
 };
 
@@ -79,70 +87,97 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
 }
 
+// Pair of work items of one CTA: items 2c and 2c+1 of one class (dense-prefix
+// query blocks first, then video query blocks, head-major), so both slots
+// have the same tile count.
+struct Pair {
+  int bh[2], qi[2];
+  bool act1;
+};
+
+__device__ __forceinline__ Pair pair_of(int cta, const Args& a) {
+  Pair p;
+  int base, count, per_head, q0;
+  if (cta < a.prefix_ctas) {
+    base = 2 * cta;
+    count = a.BH * a.pb;
+    per_head = a.pb;
+    q0 = 0;
+  } else {
+    base = 2 * (cta - a.prefix_ctas);
+    count = a.BH * a.nbv;
+    per_head = a.nbv;
+    q0 = a.pb;
+  }
+  p.act1 = base + 1 < count;
+  for (int s = 0; s < 2; ++s) {
+    const int it = min(base + s, count - 1);
+    p.bh[s] = it / per_head;
+    p.qi[s] = q0 + (it - p.bh[s] * per_head);
+  }
+  return p;
+}
+
+// Is video block j one of the listed blocks (sorted ascending in row[lo, hi))?
+__device__ __forceinline__ bool listed(const int32_t* row, int lo, int hi, int j) {
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int v = __ldg(row + mid);
+    if (v == j) return true;
+    if (v < j) lo = mid + 1; else hi = mid;
+  }
+  return false;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ks,
                   const __grid_constant__ CUtensorMap tm_vs, const Args a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t sm[];
   Ctl* ctl = reinterpret_cast<Ctl*>(sm + kOffCtl);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
   // A CTA that starts after another one recorded an expired wait does nothing
-  // (decided by one thread so that the whole CTA takes the same branch).
-  if (tid == 0)
-    ctl->skip = (a.dev_status && *reinterpret_cast<volatile int*>(a.dev_status) != 0) ? 1 : 0;
+  // (decided by one thread so that the whole CTA takes the same branch); so
+  // does one whose shared window is not 1024-byte aligned (the swizzled
+  // operand layouts need it), after recording the failure.
+  if (tid == 0) {
+    const bool bad_align = (smem_u32(sm) & 1023u) != 0;
+    if (bad_align && a.dev_status) atomicExch(a.dev_status, kErrTimeout);
+    ctl->skip = (bad_align || (a.dev_status && *reinterpret_cast<volatile int*>(a.dev_status) != 0))
+                    ? 1 : 0;
+  }
   __syncthreads();
   if (ctl->skip) return;
 
-  // Work item: dense-prefix query blocks first (they are the long ones),
-  // then video query blocks, head-major so concurrent CTAs share K/V in L2.
-  int item = blockIdx.x, bh, qi;
-  const int n_prefix_items = a.BH * a.pb;
-  if (item < n_prefix_items) {
-    bh = item / a.pb;
-    qi = item - bh * a.pb;
-  } else {
-    item -= n_prefix_items;
-    bh = item / a.nbv;
-    qi = a.pb + (item - bh * a.nbv);
-  }
-  const int32_t* idx_row = a.idx + (static_cast<size_t>(bh) * a.nb + qi) * a.kcap;
-  const int n_exact = __ldg(a.cnt + static_cast<size_t>(bh) * a.nb + qi);
-  const bool has_sum = (qi >= a.pb) && (a.k_eff < a.nbv);
+  const Pair pr = pair_of(blockIdx.x, a);
+  const bool video = pr.qi[0] >= a.pb;
+  const int n_exact = video ? a.pb + a.k_eff : a.nb;
+  const bool has_sum = video && (a.k_eff < a.nbv);
   const int u0 = a.pb / kBlock;
-  const int n_tiles = n_exact + (has_sum ? ((a.nb + kBlock - 1) / kBlock - u0) : 0);
-  const int nbw = (a.nb + 31) / 32;
+  const int T = n_exact + (has_sum ? ((a.nb + kBlock - 1) / kBlock - u0) : 0);
+  const int nslots = pr.act1 ? 2 : 1;
 
   if (tid == 0) {
-    mbar_init(&ctl->q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&ctl->k_full[s], 1);
-      mbar_init(&ctl->k_empty[s], 1);
-      mbar_init(&ctl->v_full[s], 1);
-      mbar_init(&ctl->v_empty[s], 1);
-      mbar_init(&ctl->s_full[s], 1);
-      mbar_init(&ctl->s_free[s], 128);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&ctl->full[i], 1);
+      mbar_init(&ctl->empty[i], 1);
     }
-    mbar_init(&ctl->p_full, 128);
-    mbar_init(&ctl->pv_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ctl->q_full[s], 1);
+      mbar_init(&ctl->s_full[s], 1);
+      mbar_init(&ctl->p_full[s], 128);
+      mbar_init(&ctl->o_final[s], 1);
+      mbar_init(&ctl->bias_full[s][0], 128);
+      mbar_init(&ctl->bias_full[s][1], 128);
+    }
     mbar_init(&ctl->fin, 1);
-    mbar_init(&ctl->bias_full[0], 128);
-    mbar_init(&ctl->bias_full[1], 128);
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&ctl->tmem_base, kTmemCols);
     tmem_relinquish();
-  }
-  if (has_sum) {
-    for (int w = tid; w < nbw; w += kThreads) ctl->bitmap[w] = 0u;
-    __syncthreads();
-    for (int t = a.pb + tid; t < n_exact; t += kThreads) {
-      const int j = __ldg(idx_row + t);
-      atomicOr(&ctl->bitmap[j >> 5], 1u << (j & 31));
-    }
   }
   tc_fence_before();
   __syncthreads();
@@ -150,131 +185,155 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = ctl->tmem_base;
   const WaitCtx wc{&ctl->abort_flag, a.dev_status};
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && n_tiles > 0) {
+  if (warp >= 8) {
+    reg_dealloc<kControlRegs>();
+    if (warp == kProducerWarp && lane == 0) {
+    // ---------------------------------------------------------- producer
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
-      mbar_arrive_expect_tx(&ctl->q_full, kTileBytes);
-      tma_load_3d(sm + kOffQ, &tm_q, &ctl->q_full, 0, qi * kBlock, bh);
-      tma_load_3d(sm + kOffQ + kSubBytes, &tm_q, &ctl->q_full, 64, qi * kBlock, bh);
-      int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
-      for (int t = 0; t < n_tiles; ++t) {
-        const int st = t & 1;
-        const CUtensorMap *mk, *mv;
+      for (int s = 0; s < nslots; ++s) {
+        mbar_arrive_expect_tx(&ctl->q_full[s], kTileBytes);
+        tma_load_3d(sm + kOffQ + s * kTileBytes, &tm_q, &ctl->q_full[s], 0, pr.qi[s] * kBlock,
+                    pr.bh[s]);
+        tma_load_3d(sm + kOffQ + s * kTileBytes + kSubBytes, &tm_q, &ctl->q_full[s], 64,
+                    pr.qi[s] * kBlock, pr.bh[s]);
+      }
+      int seq = 0;
+      bool ok = true;
+      // One operand tile (K or V of slot s, tile t) into the next ring stage.
+      auto emit = [&](int s, int t, bool is_v) {
+        if (!ok) return;
+        const int stage = seq % kRing;
+        if (seq >= kRing && !mbar_wait(&ctl->empty[stage], ((seq / kRing) - 1) & 1, wc)) {
+          ok = false;
+          return;
+        }
+        const CUtensorMap* m;
         int row;
         if (t < n_exact) {
-          row = __ldg(idx_row + t) * kBlock;
-          mk = &tm_k;
-          mv = &tm_v;
+          row = __ldg(a.idx + (static_cast<size_t>(pr.bh[s]) * a.nb + pr.qi[s]) * a.kcap + t) *
+                kBlock;
+          m = is_v ? &tm_v : &tm_k;
         } else {
           row = (u0 + t - n_exact) * kBlock;
-          mk = &tm_ks;
-          mv = &tm_vs;
+          m = is_v ? &tm_vs : &tm_ks;
         }
-        if (t >= 2 && !mbar_wait(&ctl->k_empty[st], ((t >> 1) - 1) & 1, wc)) break;
-        uint8_t* kd = sm + kOffK + st * kTileBytes;
-        mbar_arrive_expect_tx(&ctl->k_full[st], kTileBytes);
-        tma_load_3d(kd, mk, &ctl->k_full[st], 0, row, bh);
-        tma_load_3d(kd + kSubBytes, mk, &ctl->k_full[st], 64, row, bh);
-        k_last[st] = t;
-        if (t >= 2 && !mbar_wait(&ctl->v_empty[st], ((t >> 1) - 1) & 1, wc)) break;
-        uint8_t* vd = sm + kOffV + st * kTileBytes;
-        mbar_arrive_expect_tx(&ctl->v_full[st], kTileBytes);
-        tma_load_3d(vd, mv, &ctl->v_full[st], 0, row, bh);
-        tma_load_3d(vd + kSubBytes, mv, &ctl->v_full[st], 64, row, bh);
-        v_last[st] = t;
+        uint8_t* dst = sm + kOffRing + stage * kTileBytes;
+        mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
+        tma_load_3d(dst, m, &ctl->full[stage], 0, row, pr.bh[s]);
+        tma_load_3d(dst + kSubBytes, m, &ctl->full[stage], 64, row, pr.bh[s]);
+        ++seq;
+      };
+      for (int s = 0; s < nslots; ++s) emit(s, 0, false);
+      for (int t = 0; t < T && ok; ++t) {
+        for (int s = 0; s < nslots; ++s) {
+          emit(s, t, true);
+          if (t + 1 < T) emit(s, t + 1, false);
+        }
       }
-      // Drain: every load this thread issued has landed before the CTA exits
-      // (immediate on the normal path, where the consumer already waited).
-      mbar_wait(&ctl->q_full, 0, wc);
-      for (int s = 0; s < 2; ++s) {
-        if (k_last[s] >= 0) mbar_wait(&ctl->k_full[s], (k_last[s] >> 1) & 1, wc);
-        if (v_last[s] >= 0) mbar_wait(&ctl->v_full[s], (v_last[s] >> 1) & 1, wc);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_tiles > 0) {
+      // Drain: every issued load has landed before the CTA exits (immediate
+      // on the normal path, where the MMA warp already waited for them).
+      for (int s = 0; s < nslots; ++s) mbar_wait(&ctl->q_full[s], 0, wc);
+      for (int k = (seq > kRing ? seq - kRing : 0); k < seq; ++k)
+        mbar_wait(&ctl->full[k % kRing], (k / kRing) & 1, wc);
+    } else if (warp == kMmaWarp && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
       const uint32_t id_s = idesc_bf16_f32(128, 128, 0);
       const uint32_t id_pv = idesc_bf16_f32(128, 128, 1);
-      const uint32_t q_addr = smem_u32(sm + kOffQ);
-      const uint32_t p_addr = smem_u32(sm + kOffP);
-      bool ok = mbar_wait(&ctl->q_full, 0, wc);
-      for (int t = 0; ok && t <= n_tiles; ++t) {
-        if (t < n_tiles) {
-          const int st = t & 1;
-          if (!mbar_wait(&ctl->k_full[st], (t >> 1) & 1, wc)) break;
-          if (t >= 2 && !mbar_wait(&ctl->s_free[st], ((t >> 1) - 1) & 1, wc)) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm + kOffK + st * kTileBytes);
+      int seq = 0;
+      bool ok = true;
+      auto take = [&]() -> uint32_t {   // wait for the next ring stage
+        const int stage = seq % kRing;
+        if (!mbar_wait(&ctl->full[stage], (seq / kRing) & 1, wc)) ok = false;
+        return static_cast<uint32_t>(stage);
+      };
+      auto release = [&](uint32_t stage) {
+        mma_commit(&ctl->empty[stage]);
+        ++seq;
+      };
+      auto issue_s = [&](int s) {
+        const uint32_t stage = take();
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sm + kOffQ + s * kTileBytes);
+        const uint32_t k_addr = smem_u32(sm + kOffRing + stage * kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
-            mma_bf16_ss(tmem + kColS + st * 128, smem_desc_sw128(q_addr + off, 16, 1024),
-                        smem_desc_sw128(k_addr + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&ctl->s_full[st]);
-          mma_commit(&ctl->k_empty[st]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;
+          mma_bf16_ss(tmem + kColS + s * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+                      smem_desc_sw128(k_addr + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
         }
-        if (t >= 1) {
-          const int tp = t - 1, st = tp & 1;
-          if (!mbar_wait(&ctl->v_full[st], (tp >> 1) & 1, wc)) break;
-          if (!mbar_wait(&ctl->p_full, tp & 1, wc)) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(sm + kOffV + st * kTileBytes);
+        mma_commit(&ctl->s_full[s]);
+        release(stage);
+      };
+      auto issue_pv = [&](int s, int t) {
+        if (!mbar_wait(&ctl->p_full[s], t & 1, wc)) { ok = false; return; }
+        const uint32_t stage = take();
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sm + kOffRing + stage * kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            mma_bf16_ss(tmem + kColO,
-                        smem_desc_sw128(p_addr + (kk >> 2) * kSubBytes + (kk & 3) * 32, 16, 1024),
-                        smem_desc_sw128(v_addr + kk * 2048, kSubBytes, 1024), id_pv,
-                        (tp > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&ctl->pv_done);
-          mma_commit(&ctl->v_empty[st]);
+        for (int kk = 0; kk < 8; ++kk) {
+          mma_bf16_ts(tmem + kColO + s * 128, tmem + kColS + s * 128 + kk * 8,
+                      smem_desc_sw128(v_addr + kk * 2048, kSubBytes, 1024), id_pv,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        release(stage);
+      };
+      for (int s = 0; s < nslots && ok; ++s) {
+        if (!mbar_wait(&ctl->q_full[s], 0, wc)) ok = false;
+      }
+      for (int s = 0; s < nslots && ok; ++s) issue_s(s);
+      for (int t = 0; t < T && ok; ++t) {
+        for (int s = 0; s < nslots && ok; ++s) {
+          issue_pv(s, t);
+          if (!ok) break;
+          if (t + 1 < T) issue_s(s);
+          else mma_commit(&ctl->o_final[s]);
         }
       }
       mma_commit(&ctl->fin);
       mbar_wait(&ctl->fin, 0, wc);
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax
-    const int r = tid - 128;                       // query row within the block
-    const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = n_tiles > 0;
-    uint8_t* prow = sm + kOffP + r * 128;
+  } else {
+    reg_alloc<kSoftmaxRegs>();
+    // ---------------------------------------------------------- softmax
+    const int s = warp >> 2;                       // slot
+    const int r = tid & 127;                       // query row within the block
+    const bool active = s < nslots;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + kColS + s * 128;
+    const uint32_t o_col = tmem + lane_base + kColO + s * 128;
+    const int bh = pr.bh[s], qi = pr.qi[s];
+    const int32_t* idx_row = a.idx + (static_cast<size_t>(bh) * a.nb + qi) * a.kcap;
     const float* bias_h = a.bias + static_cast<size_t>(bh) * a.nb;
-    float* ctl_bias = &ctl->bias_stage[0][0];
-    for (int t = 0; ok && t < n_tiles; ++t) {
-      const int sb = t & 1;
+    float* stage_buf = &ctl->bias_stage[s][0][0];
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = active;
+    for (int t = 0; ok && t < T; ++t) {
       if (t >= n_exact) {
         // Stage summary tile v's bias in log2 units, -inf where the column is
         // a listed block, a prefix block or past the last block.  Buffer v&1
-        // is free again: every reader of its previous use (tile t-2) finished
-        // that tile before PV(t-2) could run, and this thread waited for
-        // PV(t-2) in tile t-1.
+        // is free again: all 128 threads finished tile t-2 before PV(t-2)
+        // could run, and this thread saw S(t-1), issued after PV(t-2).
         const int v = t - n_exact;
         const int j = (u0 + v) * kBlock + r;
         float b = -INFINITY;
-        if (j >= a.pb && j < a.nb && !((ctl->bitmap[j >> 5] >> (j & 31)) & 1u))
+        if (j >= a.pb && j < a.nb && !listed(idx_row, a.pb, n_exact, j))
           b = __ldg(bias_h + j) * kLog2e;
-        ctl_bias[(v & 1) * 128 + r] = b;
-        mbar_arrive(&ctl->bias_full[v & 1]);
-        if (!warp_wait(&ctl->bias_full[v & 1], (v >> 1) & 1, wc)) { ok = false; break; }
+        stage_buf[(v & 1) * 128 + r] = b;
+        mbar_arrive(&ctl->bias_full[s][v & 1]);
+        if (!warp_wait(&ctl->bias_full[s][v & 1], (v >> 1) & 1, wc)) { ok = false; break; }
       }
-      if (!warp_wait(&ctl->s_full[sb], (t >> 1) & 1, wc)) { ok = false; break; }
+      if (!warp_wait(&ctl->s_full[s], t & 1, wc)) { ok = false; break; }
       tc_fence_after();
       float x[128];
-      const uint32_t sa = tmem + lane_base + kColS + sb * 128;
-      BSA_TMEM_LD_32F(sa, x);
-      BSA_TMEM_LD_32F(sa + 32, x + 32);
-      BSA_TMEM_LD_32F(sa + 64, x + 64);
-      BSA_TMEM_LD_32F(sa + 96, x + 96);
+      BSA_TMEM_LD_32F(s_col, x);
+      BSA_TMEM_LD_32F(s_col + 32, x + 32);
+      BSA_TMEM_LD_32F(s_col + 64, x + 64);
+      BSA_TMEM_LD_32F(s_col + 96, x + 96);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&ctl->s_free[sb]);
 
       if (t < n_exact) {
         const int j = __ldg(idx_row + t);
@@ -282,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 128; ++c) x[c] = (c < ncols) ? x[c] * a.scale_log2 : -INFINITY;
       } else {
-        const float4* bb4 = reinterpret_cast<const float4*>(ctl_bias + ((t - n_exact) & 1) * 128);
+        const float4* bb4 = reinterpret_cast<const float4*>(stage_buf + ((t - n_exact) & 1) * 128);
 #pragma unroll
         for (int c4 = 0; c4 < 32; ++c4) {
           const float4 b = bb4[c4];
@@ -298,57 +357,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool need = mx > m_run + kRescaleThreshold;
       const float m_new = need ? mx : m_run;
       const float alpha = need ? fast_exp2(m_run - m_new) : 1.0f;
-      if (t > 0) {
-        // PV(t-1) done: the P buffer is free and O is stable
-        if (!warp_wait(&ctl->pv_done, (t - 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-      }
-      float rs = 0.f;
-#pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = fast_exp2(x[c8 * 8 + 2 * e] - m_new);
-          const float p1 = fast_exp2(x[c8 * 8 + 2 * e + 1] - m_new);
-          rs += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        const int sub = c8 >> 3, cc = c8 & 7;
-        *reinterpret_cast<uint4*>(prow + sub * kSubBytes + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
+      // O_s is stable here: PV_s(t-1) was issued before S_s(t) and the MMAs
+      // of one thread complete in order.
       if (t > 0 && __any_sync(0xffffffffu, need)) {
-        const uint32_t oa = tmem + lane_base + kColO;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float o[32];
-          BSA_TMEM_LD_32F(oa + q * 32, o);
+          BSA_TMEM_LD_32F(o_col + q * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          BSA_TMEM_ST_32(oa + q * 32, reinterpret_cast<uint32_t*>(o));
+          BSA_TMEM_ST_32(o_col + q * 32, reinterpret_cast<uint32_t*>(o));
         }
-        tmem_wait_st();
       }
+      float rs = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = fast_exp2(x[64 * h + 2 * e] - m_new);
+          const float p1 = fast_exp2(x[64 * h + 2 * e + 1] - m_new);
+          rs += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        BSA_TMEM_ST_32(s_col + 32 * h, pk);
+      }
+      tmem_wait_st();
       m_run = m_new;
       l_run = l_run * alpha + rs;
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&ctl->p_full);
+      mbar_arrive(&ctl->p_full[s]);
     }
-    // ---------------------------------------------------------- epilogue
-    if (ok && warp_wait(&ctl->pv_done, (n_tiles - 1) & 1, wc)) {
+    // -------------------------------------------------------- epilogue
+    if (ok && warp_wait(&ctl->o_final[s], 0, wc)) {
       tc_fence_after();
       const int qrow = qi * kBlock + r;
       const bool live = qrow < a.N;
       const float inv_l = 1.f / l_run;
       uint4* orow = reinterpret_cast<uint4*>(a.O + (static_cast<size_t>(bh) * a.N + qrow) * kDim);
-      const uint32_t oa = tmem + lane_base + kColO;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float o[32];
-        BSA_TMEM_LD_32F(oa + q * 32, o);
+        BSA_TMEM_LD_32F(o_col + q * 32, o);
         tmem_wait_ld();
         if (live) {
 #pragma unroll
@@ -367,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -391,26 +442,24 @@ __global__ void expired_wait_kernel(int* dev_status, uint64_t timeout_ns) {
 
 }  // namespace
 
-static size_t attend_smem_bytes(int nb) {
-  // bitmap words plus 4 spare words, so no guarded read can leave the allocation
-  return 1024 + kOffCtl + sizeof(Ctl) + sizeof(uint32_t) * ((nb + 31) / 32 + 4);
-}
-
 cudaError_t launch_attend(const Shape& s, const AttendMaps& maps, const int32_t* idx,
                           const int32_t* cnt, const float* bias, void* O, float* lse,
                           cudaStream_t st) {
+  // Tile counts follow from (pb, k_eff, nb): bsa_select lists pb + k_eff
+  // blocks for every video query block and all nb for a prefix block.
+  (void)cnt;
+  constexpr size_t smem = kOffCtl + sizeof(Ctl);
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         227 * 1024);
+    cudaError_t e =
+        cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   Args a;
   a.idx = idx;
-  a.cnt = cnt;
   a.bias = bias;
   a.O = static_cast<__nv_bfloat16*>(O);
   a.lse = lse;
@@ -422,10 +471,10 @@ cudaError_t launch_attend(const Shape& s, const AttendMaps& maps, const int32_t*
   a.k_eff = s.k_eff;
   a.kcap = s.kcap;
   a.BH = s.B * s.H;
+  a.prefix_ctas = (a.BH * s.pb + 1) / 2;
   a.scale_log2 = kLog2e * 0.088388347648318440550f;
-  const int grid = a.BH * s.nb;
-  attend_kernel<<<grid, kThreads, attend_smem_bytes(s.nb), st>>>(maps.q, maps.k, maps.v, maps.ks,
-                                                                 maps.vs, a);
+  const int grid = a.prefix_ctas + (a.BH * s.nbv + 1) / 2;
+  attend_kernel<<<grid, kThreads, smem, st>>>(maps.q, maps.k, maps.v, maps.ks, maps.vs, a);
   return cudaGetLastError();
 }
 
