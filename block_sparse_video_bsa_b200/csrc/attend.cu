@@ -63,7 +63,7 @@ struct Ctl {
   uint64_t full[kRing], empty[kRing];
   uint64_t q_full[2];
   uint64_t s_full[2], p_full[2], o_final[2];
-  uint64_t bias_full[2][2];
+  uint64_t bias_full[2][2], bias_empty[2][2];
   uint64_t fin;
   uint32_t tmem_base;
   int abort_flag;
@@ -168,8 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->s_full[s], 1);
       mbar_init(&ctl->p_full[s], 128);
       mbar_init(&ctl->o_final[s], 1);
-      mbar_init(&ctl->bias_full[s][0], 128);
-      mbar_init(&ctl->bias_full[s][1], 128);
+      mbar_init(&ctl->bias_full[s][0], 32);
+      mbar_init(&ctl->bias_full[s][1], 32);
+      mbar_init(&ctl->bias_empty[s][0], 128);
+      mbar_init(&ctl->bias_empty[s][1], 128);
     }
     mbar_init(&ctl->fin, 1);
     ctl->abort_flag = 0;
@@ -295,6 +297,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(&ctl->fin);
       mbar_wait(&ctl->fin, 0, wc);
+    } else if (warp >= 10 && has_sum && warp - 10 < nslots) {
+    // ---------------------------------------------------------- bias stager
+      // Warp 10 + s stages, for each summary tile v of slot s, the 128 biases
+      // in log2 units with -inf where the column is a listed block, a prefix
+      // block or past the last block (listed: binary search of the sorted
+      // idx row), double buffered against the slot's softmax warps.
+      const int s = warp - 10;
+      const int32_t* idx_row = a.idx + (static_cast<size_t>(pr.bh[s]) * a.nb + pr.qi[s]) * a.kcap;
+      const float* bias_h = a.bias + static_cast<size_t>(pr.bh[s]) * a.nb;
+      for (int v = 0; v < T - n_exact; ++v) {
+        if (v >= 2 && !warp_wait(&ctl->bias_empty[s][v & 1], ((v >> 1) - 1) & 1, wc)) break;
+        float* dst = &ctl->bias_stage[s][v & 1][0];
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          const int c = lane + 32 * q;
+          const int j = (u0 + v) * kBlock + c;
+          float b = -INFINITY;
+          if (j >= a.pb && j < a.nb && !listed(idx_row, a.pb, n_exact, j))
+            b = __ldg(bias_h + j) * kLog2e;
+          dst[c] = b;
+        }
+        mbar_arrive(&ctl->bias_full[s][v & 1]);
+      }
     }
   } else {
     reg_alloc<kSoftmaxRegs>();
@@ -307,25 +332,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_col = tmem + lane_base + kColO + s * 128;
     const int bh = pr.bh[s], qi = pr.qi[s];
     const int32_t* idx_row = a.idx + (static_cast<size_t>(bh) * a.nb + qi) * a.kcap;
-    const float* bias_h = a.bias + static_cast<size_t>(bh) * a.nb;
-    float* stage_buf = &ctl->bias_stage[s][0][0];
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = active;
+    // Only the last listed block can be the ragged last block (lists are
+    // ascending and nb-1 is the largest index): find it once.
+    int ragged_t = -1, ragged_cols = kBlock;
+    if (active && (a.N % kBlock) != 0 && __ldg(idx_row + n_exact - 1) == a.nb - 1) {
+      ragged_t = n_exact - 1;
+      ragged_cols = a.N - (a.nb - 1) * kBlock;
+    }
     for (int t = 0; ok && t < T; ++t) {
-      if (t >= n_exact) {
-        // Stage summary tile v's bias in log2 units, -inf where the column is
-        // a listed block, a prefix block or past the last block.  Buffer v&1
-        // is free again: all 128 threads finished tile t-2 before PV(t-2)
-        // could run, and this thread saw S(t-1), issued after PV(t-2).
-        const int v = t - n_exact;
-        const int j = (u0 + v) * kBlock + r;
-        float b = -INFINITY;
-        if (j >= a.pb && j < a.nb && !listed(idx_row, a.pb, n_exact, j))
-          b = __ldg(bias_h + j) * kLog2e;
-        stage_buf[(v & 1) * 128 + r] = b;
-        mbar_arrive(&ctl->bias_full[s][v & 1]);
-        if (!warp_wait(&ctl->bias_full[s][v & 1], (v >> 1) & 1, wc)) { ok = false; break; }
-      }
+      const bool exact = t < n_exact;
+      const int v = t - n_exact;   // summary tile index when !exact
       if (!warp_wait(&ctl->s_full[s], t & 1, wc)) { ok = false; break; }
       tc_fence_after();
       float x[128];
@@ -335,57 +353,78 @@ __global__ void __launch_bounds__(kThreads, 1)
       BSA_TMEM_LD_32F(s_col + 96, x + 96);
       tmem_wait_ld();
 
-      if (t < n_exact) {
-        const int j = __ldg(idx_row + t);
-        const int ncols = min(kBlock, a.N - j * kBlock);
+      // Exact tiles keep raw scores (the scale is folded into the exponent's
+      // FMA; scale > 0 so max commutes with it); summary tiles become
+      // logits in log2 units with the staged bias / mask.
+      float2 mul = make_float2(a.scale_log2, a.scale_log2);
+      if (exact) {
+        if (t == ragged_t) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = (c < ncols) ? x[c] * a.scale_log2 : -INFINITY;
+          for (int c = 0; c < 128; ++c)
+            if (c >= ragged_cols) x[c] = -INFINITY;
+        }
       } else {
-        const float4* bb4 = reinterpret_cast<const float4*>(stage_buf + ((t - n_exact) & 1) * 128);
+        if (!warp_wait(&ctl->bias_full[s][v & 1], (v >> 1) & 1, wc)) { ok = false; break; }
+        const float4* bb4 = reinterpret_cast<const float4*>(&ctl->bias_stage[s][v & 1][0]);
 #pragma unroll
         for (int c4 = 0; c4 < 32; ++c4) {
           const float4 b = bb4[c4];
-          x[4 * c4 + 0] = fmaf(x[4 * c4 + 0], a.scale_log2, b.x);
-          x[4 * c4 + 1] = fmaf(x[4 * c4 + 1], a.scale_log2, b.y);
-          x[4 * c4 + 2] = fmaf(x[4 * c4 + 2], a.scale_log2, b.z);
-          x[4 * c4 + 3] = fmaf(x[4 * c4 + 3], a.scale_log2, b.w);
+          const float2 y0 = fma2(make_float2(x[4 * c4], x[4 * c4 + 1]), mul, make_float2(b.x, b.y));
+          const float2 y1 = fma2(make_float2(x[4 * c4 + 2], x[4 * c4 + 3]), mul, make_float2(b.z, b.w));
+          x[4 * c4] = y0.x; x[4 * c4 + 1] = y0.y; x[4 * c4 + 2] = y1.x; x[4 * c4 + 3] = y1.y;
         }
+        mbar_arrive(&ctl->bias_empty[s][v & 1]);
+        mul = make_float2(1.f, 1.f);
       }
-      float mx = -INFINITY;
+      float mp[8];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      for (int k = 0; k < 8; ++k) mp[k] = x[k];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * mul.x;
       const bool need = mx > m_run + kRescaleThreshold;
       const float m_new = need ? mx : m_run;
       const float alpha = need ? fast_exp2(m_run - m_new) : 1.0f;
       // O_s is stable here: PV_s(t-1) was issued before S_s(t) and the MMAs
       // of one thread complete in order.
       if (t > 0 && __any_sync(0xffffffffu, need)) {
+        const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float o[32];
           BSA_TMEM_LD_32F(o_col + q * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          for (int e = 0; e < 16; ++e) {
+            const float2 r2 = mul2(make_float2(o[2 * e], o[2 * e + 1]), al2);
+            o[2 * e] = r2.x;
+            o[2 * e + 1] = r2.y;
+          }
           BSA_TMEM_ST_32(o_col + q * 32, reinterpret_cast<uint32_t*>(o));
         }
       }
-      float rs = 0.f;
+      // p = 2^(x * mul - m_new); four packed partial row sums.
+      const float2 off = make_float2(-m_new, -m_new);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float p0 = fast_exp2(x[64 * h + 2 * e] - m_new);
-          const float p1 = fast_exp2(x[64 * h + 2 * e + 1] - m_new);
-          rs += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          const float2 y = fma2(make_float2(x[64 * h + 2 * e], x[64 * h + 2 * e + 1]), mul, off);
+          const float2 p2 = make_float2(fast_exp2(y.x), fast_exp2(y.y));
+          acc[e & 3] = add2(acc[e & 3], p2);
+          pk[e] = pack_bf16x2(p2.x, p2.y);
         }
         BSA_TMEM_ST_32(s_col + 32 * h, pk);
       }
+      const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+      const float2 a4 = add2(a01, a23);
       tmem_wait_st();
       m_run = m_new;
-      l_run = l_run * alpha + rs;
+      l_run = l_run * alpha + (a4.x + a4.y);
       tc_fence_before();
       mbar_arrive(&ctl->p_full[s]);
     }
