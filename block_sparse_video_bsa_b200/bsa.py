@@ -79,7 +79,7 @@ def header_functions() -> list:
     """Names of the functions include/bsa.h declares."""
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bsa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(bsa_[a-z0-9_]+)\s*\(", text)))
 
 
 def status_string(status: int) -> str:
