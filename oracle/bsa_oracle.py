@@ -172,7 +172,7 @@ def select_blocks(S: np.ndarray, top_k: int, prefix_blocks: int):
 
 
 def attend(Q: np.ndarray, K: np.ndarray, V: np.ndarray, lists, ksum, vsum, bias,
-           prefix_blocks: int, block: int = BLOCK):
+           prefix_blocks: int, block: int = BLOCK, query_blocks=None):
     """Exact branch + compressed branch, one softmax per query row.
 
     For query row t in block i the logits are
@@ -180,7 +180,8 @@ def attend(Q: np.ndarray, K: np.ndarray, V: np.ndarray, lists, ksum, vsum, bias,
       { q_t . k~_j / sqrt(d) + bias_j : j >= pb, j not in E_i }      (summaries)
     and O_t = softmax(logits) @ [V rows ; v~ rows].  Dense-prefix query rows
     have every block in E_i and therefore no summary rows.  Also returns
-    lse_t = log sum exp(logits) (natural log).
+    lse_t = log sum exp(logits) (natural log).  ``query_blocks`` optionally
+    restricts the work to those query blocks (other rows are left at 0).
     """
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
@@ -193,6 +194,8 @@ def attend(Q: np.ndarray, K: np.ndarray, V: np.ndarray, lists, ksum, vsum, bias,
     O = np.zeros((N, V.shape[1]))
     lse = np.zeros(N)
     for i, (a, b) in enumerate(bounds):
+        if query_blocks is not None and i not in query_blocks:
+            continue
         E = list(lists[i])
         tok = np.concatenate([np.arange(*bounds[j]) for j in E])
         logits = (Q[a:b] @ K[tok].T) * scale
@@ -213,11 +216,12 @@ def attend(Q: np.ndarray, K: np.ndarray, V: np.ndarray, lists, ksum, vsum, bias,
 
 
 def forward_head(Q, K, V, top_k: int, prefix: int = 0, variant: str = "anchor",
-                 block: int = BLOCK):
+                 block: int = BLOCK, query_blocks=None):
     """The whole path for one (batch, head) slice: pool, summarize, select, attend.
 
     Q, K, V are [N, d] arrays (any float type; widened to float64).  Returns a
     dict with every intermediate so tests can compare stage by stage.
+    ``query_blocks`` restricts only the attention step (see ``attend``).
     """
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
@@ -234,7 +238,7 @@ def forward_head(Q, K, V, top_k: int, prefix: int = 0, variant: str = "anchor",
     ksum, vsum, bias = block_summaries(K, V, qbar, variant, block)
     S = block_scores(qpool, kpool)
     lists = select_blocks(S, top_k, pb)
-    O, lse = attend(Q, K, V, lists, ksum, vsum, bias, pb, block)
+    O, lse = attend(Q, K, V, lists, ksum, vsum, bias, pb, block, query_blocks)
     return dict(qpool=qpool, kpool=kpool, anchor=qbar, ksum=ksum, vsum=vsum,
                 bias=bias, scores=S, lists=lists, O=O, lse=lse)
 
@@ -252,7 +256,8 @@ def forward(Q, K, V, top_k: int, prefix: int = 0, variant: str = "anchor",
     return O
 
 
-def effective_pairs(N: int, lists, prefix_blocks: int, block: int = BLOCK) -> int:
+def effective_pairs(N: int, lists, prefix_blocks: int, block: int = BLOCK,
+                    query_blocks=None) -> int:
     """Computed (query, key-or-summary) pairs of one head, masked columns excluded.
 
     Exact pairs count the real tokens of each listed block; summary pairs
@@ -263,6 +268,8 @@ def effective_pairs(N: int, lists, prefix_blocks: int, block: int = BLOCK) -> in
     nb = len(bounds)
     total = 0
     for i, (a, b) in enumerate(bounds):
+        if query_blocks is not None and i not in query_blocks:
+            continue
         rows = b - a
         exact = sum(bounds[j][1] - bounds[j][0] for j in lists[i])
         summ = 0 if i < prefix_blocks else (nb - prefix_blocks) - (len(lists[i]) - prefix_blocks)
