@@ -255,8 +255,6 @@ int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK, const 
   int rc = shape_of(p, &s);
   if (rc) return rc;
   if (!hQ || !hK || !hV || !hO) return BSA_ERR_INVALID;
-  const size_t bytes = static_cast<size_t>(s.B) * s.H * s.N * 128 * 2;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Validate the device side before the first copy so an error enqueues nothing.
   if (!dQ || !dK || !dV || !dO || !workspace) return BSA_ERR_INVALID;
   if (workspace_bytes < carve(s, nullptr, nullptr)) return BSA_ERR_INVALID;
@@ -264,17 +262,88 @@ int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK, const 
       !aligned(workspace, 256) || (dlse && !aligned(dlse, 4)))
     return BSA_ERR_ALIGN;
   if ((rc = check_device())) return rc;
-  if (cudaMemcpyAsync(dQ, hQ, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(dK, hK, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(dV, hV, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+
+  // Pipeline over chunks of (b, h) slices (every slice is independent):
+  // host->device copies on one helper stream, the forward on the caller's
+  // stream, device->host copies on another helper stream, ordered by events.
+  // Copies of chunk c+1 overlap the forward of chunk c, and the two copy
+  // directions overlap each other.  The helper streams and events are made
+  // per call and released when their work is done; the caller's stream
+  // waits for the last copy, so synchronising it covers everything.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = s.B * s.H;
+  const int nchunk = BH < 8 ? BH : 8;
+  const int per = (BH + nchunk - 1) / nchunk;
+  const size_t slice = static_cast<size_t>(s.N) * 128 * 2;     // bytes of one (b, h) slice
+  const size_t lslice = static_cast<size_t>(s.N) * 4;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_done = nullptr, ev_in[8] = {}, ev_comp[8] = {};
+  auto cleanup = [&]() {
+    for (int c = 0; c < 8; ++c) {
+      if (ev_in[c]) cudaEventDestroy(ev_in[c]);
+      if (ev_comp[c]) cudaEventDestroy(ev_comp[c]);
+    }
+    if (ev_start) cudaEventDestroy(ev_start);
+    if (ev_done) cudaEventDestroy(ev_done);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+  };
+  bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming) == cudaSuccess;
+  for (int c = 0; ok && c < nchunk; ++c)
+    ok = cudaEventCreateWithFlags(&ev_in[c], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&ev_comp[c], cudaEventDisableTiming) == cudaSuccess;
+  // helper streams start after earlier work on the caller's stream
+  ok = ok && cudaEventRecord(ev_start, st) == cudaSuccess &&
+       cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
+  if (!ok) {
+    cleanup();
     return BSA_ERR_CUDA;
-  if ((rc = bsa_forward(p, dQ, dK, dV, dO, dlse, workspace, workspace_bytes, stream))) return rc;
-  if (cudaMemcpyAsync(hO, dO, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return BSA_ERR_CUDA;
-  if (hlse && dlse &&
-      cudaMemcpyAsync(hlse, dlse, static_cast<size_t>(s.B) * s.H * s.N * 4, cudaMemcpyDeviceToHost,
-                      st) != cudaSuccess)
-    return BSA_ERR_CUDA;
-  return BSA_OK;
+  }
+  auto off = [](const void* base, size_t bytes) {
+    return static_cast<const char*>(base) + bytes;
+  };
+  for (int c = 0; c < nchunk && rc == BSA_OK; ++c) {
+    const int bh0 = c * per;
+    const int nbh = (BH - bh0) < per ? (BH - bh0) : per;
+    if (nbh <= 0) break;
+    const size_t o = static_cast<size_t>(bh0) * slice, bytes = static_cast<size_t>(nbh) * slice;
+    char* q = static_cast<char*>(dQ) + o;
+    char* k = static_cast<char*>(dK) + o;
+    char* v = static_cast<char*>(dV) + o;
+    char* out = static_cast<char*>(dO) + o;
+    float* l = dlse ? dlse + static_cast<size_t>(bh0) * s.N : nullptr;
+    if (cudaMemcpyAsync(q, off(hQ, o), bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(k, off(hK, o), bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(v, off(hV, o), bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaEventRecord(ev_in[c], s_in) != cudaSuccess ||
+        cudaStreamWaitEvent(st, ev_in[c], 0) != cudaSuccess) {
+      rc = BSA_ERR_CUDA;
+      break;
+    }
+    bsa_params sub = *p;
+    sub.B = 1;
+    sub.H = nbh;
+    if ((rc = bsa_forward(&sub, q, k, v, out, l, workspace, workspace_bytes, stream))) break;
+    if (cudaEventRecord(ev_comp[c], st) != cudaSuccess ||
+        cudaStreamWaitEvent(s_out, ev_comp[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<char*>(hO) + o, out, bytes, cudaMemcpyDeviceToHost, s_out) !=
+            cudaSuccess ||
+        (hlse && l &&
+         cudaMemcpyAsync(hlse + static_cast<size_t>(bh0) * s.N, l, nbh * lslice,
+                         cudaMemcpyDeviceToHost, s_out) != cudaSuccess)) {
+      rc = BSA_ERR_CUDA;
+      break;
+    }
+  }
+  // the caller's stream waits for the last copy back
+  if (cudaEventRecord(ev_done, s_out) != cudaSuccess || cudaStreamWaitEvent(st, ev_done, 0) != cudaSuccess)
+    rc = rc ? rc : BSA_ERR_CUDA;
+  cleanup();
+  return rc;
 }
 
 const char* bsa_status_string(int status) {

@@ -142,11 +142,18 @@ int bsa_forward(const bsa_params* p, const void* Q, const void* K, const void* V
                 void* O, float* lse, void* workspace, size_t workspace_bytes,
                 void* stream);
 
-/* bsa_forward from HOST buffers: copies hQ, hK, hV (bf16 [B,H,N,D], pinned
- * for asynchronous copies) to the caller's device buffers dQ, dK, dV with one
- * cudaMemcpyAsync each, runs bsa_forward, and copies dO back to hO (and dlse
- * to hlse when both are non-NULL), all on `stream`.  Returns after enqueueing;
- * synchronise the stream before reading hO. */
+/* bsa_forward from HOST buffers.  hQ, hK, hV (bf16 [B,H,N,D]) are copied to
+ * the caller's device buffers dQ, dK, dV, the forward runs, and dO is copied
+ * back to hO (and dlse to hlse when both are non-NULL).  The work is
+ * pipelined over up to 8 chunks of (b, h) slices: the host->device copies
+ * (one cudaMemcpyAsync per tensor and chunk) run on a helper stream, the
+ * forward of each chunk on `stream`, the copies back on a second helper
+ * stream, ordered by events, so copies overlap compute and each other.
+ * Host buffers must be pinned for the copies to be asynchronous.  The helper
+ * streams / events are created per call and released once their work is
+ * done; `stream` waits for the last copy, so synchronising `stream` covers
+ * the whole call.  Returns after enqueueing.  On BSA_ERR_CUDA part of the
+ * work may already be enqueued. */
 int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK,
                      const void* hV, void* hO, float* hlse, void* dQ, void* dK,
                      void* dV, void* dO, float* dlse, void* workspace,
