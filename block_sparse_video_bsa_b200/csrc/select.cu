@@ -3,13 +3,18 @@
 //
 // One CTA per (tile of R query blocks, head), 256 threads:
 //  1. scores  S_ij = qpool_i . kpool_j / sqrt(128) in fp32 for every video
-//     key block j >= pb, kept in shared memory (never written to HBM);
-//     128-term dot products summed in a fixed order (deterministic).
+//     key block j >= pb, kept in shared memory (never written to HBM).  The
+//     pooled keys stream through shared memory 32 blocks at a time
+//     (coalesced 16-byte loads, rows padded against bank conflicts); each
+//     thread forms the dot products of two query blocks with one key block
+//     with packed fp32x2 FMAs (even and odd dimensions in two partial sums,
+//     added at the end; a fixed order, so the result is deterministic).
 //  2. one warp per query block finds the k_eff-th largest score as a 32-bit
 //     order-preserving key by bitwise binary search (32 count passes,
-//     __reduce_add_sync per pass), then emits, in ascending j, every block
-//     above that key plus the lowest-index blocks equal to it -- exactly
-//     "score descending, ties to the lower index".
+//     __reduce_add_sync per pass, the row's keys held in registers), then
+//     emits, in ascending j, every block above that key plus the
+//     lowest-index blocks equal to it -- exactly "score descending, ties to
+//     the lower index".
 // Dense-prefix query blocks (i < pb) list every block.
 #include "bsa_device.cuh"
 #include "bsa_kernels.h"
@@ -19,17 +24,96 @@ namespace bsa {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kMaxRows = 8;
+constexpr int kChunk = 32;               // key blocks per shared-memory chunk
+constexpr int kPad = kDim + 4;           // padded row of 132 floats
 
+// Top-k of one row of nbv scores (in shared memory) by warp `lane`s; the keys
+// are copied to registers (kPerLane per lane, nbv <= 32 * kPerLane).
+template <int kPerLane>
+__device__ __forceinline__ void topk_row(const float* srow, int nbv, int k_eff, int pb,
+                                         int32_t* row, int lane) {
+  uint32_t key[kPerLane];
+#pragma unroll
+  for (int e = 0; e < kPerLane; ++e) {
+    const int j = lane + 32 * e;
+    key[e] = (j < nbv) ? orderable_key(srow[j]) : 0u;   // 0 is below every real key
+  }
+  // k_eff-th largest key T: largest T with #{key >= T} >= k_eff.
+  uint32_t T = 0;
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t cand = T | (1u << b);
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < kPerLane; ++e) c += (key[e] >= cand) ? 1 : 0;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (c >= k_eff) T = cand;
+  }
+  int gt = 0;
+#pragma unroll
+  for (int e = 0; e < kPerLane; ++e) gt += (key[e] > T) ? 1 : 0;
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  const int need_eq = k_eff - gt;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int out = 0, eq_seen = 0;
+#pragma unroll
+  for (int e = 0; e < kPerLane; ++e) {
+    if (32 * e >= nbv) break;
+    const int j = lane + 32 * e;
+    const bool valid = j < nbv;
+    const bool is_gt = valid && key[e] > T;
+    const bool is_eq = valid && key[e] == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+    const bool sel = is_gt || (is_eq && (eq_seen + __popc(eqm & lt_mask)) < need_eq);
+    const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+    if (sel) row[pb + out + __popc(selm & lt_mask)] = pb + j;
+    out += __popc(selm);
+    eq_seen += __popc(eqm);
+  }
+}
+
+// Same selection for rows too long to keep in registers (keys re-read from
+// shared memory on every pass).
+__device__ __forceinline__ void topk_row_smem(const float* srow, int nbv, int k_eff, int pb,
+                                              int32_t* row, int lane) {
+  uint32_t T = 0;
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t cand = T | (1u << b);
+    int c = 0;
+    for (int j = lane; j < nbv; j += 32) c += (orderable_key(srow[j]) >= cand) ? 1 : 0;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (c >= k_eff) T = cand;
+  }
+  int gt = 0;
+  for (int j = lane; j < nbv; j += 32) gt += (orderable_key(srow[j]) > T) ? 1 : 0;
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  const int need_eq = k_eff - gt;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int out = 0, eq_seen = 0;
+  for (int base = 0; base < nbv; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = (j < nbv) ? orderable_key(srow[j]) : 0u;
+    const bool is_gt = (j < nbv) && (u > T);
+    const bool is_eq = (j < nbv) && (u == T);
+    const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+    const bool sel = is_gt || (is_eq && (eq_seen + __popc(eqm & lt_mask)) < need_eq);
+    const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+    if (sel) row[pb + out + __popc(selm & lt_mask)] = pb + j;
+    out += __popc(selm);
+    eq_seen += __popc(eqm);
+  }
+}
+
+template <int kPerLane>   // 0 = keys stay in shared memory
 __global__ void __launch_bounds__(kThreads) select_kernel(const float* __restrict__ qpool,
                                                           const float* __restrict__ kpool,
                                                           int32_t* __restrict__ idx,
                                                           int32_t* __restrict__ cnt, int nb, int pb,
                                                           int k_eff, int kcap, int R, float scale) {
   extern __shared__ float smem[];
-  float* qp = smem;                 // [R][128]
-  float* sc = smem + R * kDim;      // [R][nbv]
   const int nbv = nb - pb;
+  float* qp = smem;                          // [R][kPad]
+  float* kc = qp + R * kPad;                 // [kChunk][kPad]
+  float* sc = kc + kChunk * kPad;            // [R][nbv]
   const size_t bh = blockIdx.y;
   const int i0 = blockIdx.x * R;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -38,34 +122,42 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float* __restric
   for (int r = 0; r < R; ++r) any_video |= (i0 + r >= pb && i0 + r < nb);
 
   if (any_video) {
-    for (int e = tid; e < R * kDim; e += kThreads) {
-      const int r = e / kDim, d = e % kDim;
+    for (int e = tid; e < R * (kDim / 4); e += kThreads) {
+      const int r = e / (kDim / 4), d4 = e % (kDim / 4);
       const int i = min(i0 + r, nb - 1);
-      qp[e] = __ldg(qpool + (bh * nb + i) * kDim + d);
+      *reinterpret_cast<float4*>(qp + r * kPad + 4 * d4) =
+          __ldg(reinterpret_cast<const float4*>(qpool + (bh * nb + i) * kDim) + d4);
     }
-    __syncthreads();
-    for (int jj = tid; jj < nbv; jj += kThreads) {
-      const float4* kp = reinterpret_cast<const float4*>(kpool + (bh * nb + pb + jj) * kDim);
-      float acc[kMaxRows];
-#pragma unroll
-      for (int r = 0; r < kMaxRows; ++r) acc[r] = 0.f;
-#pragma unroll 4
-      for (int d4 = 0; d4 < kDim / 4; ++d4) {
-        const float4 k4 = __ldg(kp + d4);
-#pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) {
-          if (r < R) {
-            const float4 q4 = *reinterpret_cast<const float4*>(qp + r * kDim + d4 * 4);
-            acc[r] = fmaf(q4.x, k4.x, acc[r]);
-            acc[r] = fmaf(q4.y, k4.y, acc[r]);
-            acc[r] = fmaf(q4.z, k4.z, acc[r]);
-            acc[r] = fmaf(q4.w, k4.w, acc[r]);
-          }
-        }
+    // thread -> (query-block pair rp, key k of the chunk); R/2 pairs x 32 keys
+    const int pairs = R / 2;
+    const int rp = tid / kChunk, kk = tid % kChunk;
+    for (int c0 = 0; c0 < nbv; c0 += kChunk) {
+      __syncthreads();   // previous chunk fully used (and qp written, first time)
+      const int rows = min(kChunk, nbv - c0);
+      for (int e = tid; e < rows * (kDim / 4); e += kThreads) {
+        const int r = e / (kDim / 4), d4 = e % (kDim / 4);
+        *reinterpret_cast<float4*>(kc + r * kPad + 4 * d4) = __ldg(
+            reinterpret_cast<const float4*>(kpool + (bh * nb + pb + c0 + r) * kDim) + d4);
       }
-#pragma unroll
-      for (int r = 0; r < kMaxRows; ++r)
-        if (r < R) sc[r * nbv + jj] = acc[r] * scale;
+      __syncthreads();
+      if (rp < pairs && kk < rows) {
+        const float* q0 = qp + (2 * rp) * kPad;
+        const float* q1 = q0 + kPad;
+        const float* kr = kc + kk * kPad;
+        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll 8
+        for (int d4 = 0; d4 < kDim / 4; ++d4) {
+          const float4 k4 = *reinterpret_cast<const float4*>(kr + 4 * d4);
+          const float4 x0 = *reinterpret_cast<const float4*>(q0 + 4 * d4);
+          const float4 x1 = *reinterpret_cast<const float4*>(q1 + 4 * d4);
+          a0 = fma2(make_float2(x0.x, x0.y), make_float2(k4.x, k4.y), a0);
+          a0 = fma2(make_float2(x0.z, x0.w), make_float2(k4.z, k4.w), a0);
+          a1 = fma2(make_float2(x1.x, x1.y), make_float2(k4.x, k4.y), a1);
+          a1 = fma2(make_float2(x1.z, x1.w), make_float2(k4.z, k4.w), a1);
+        }
+        sc[(2 * rp) * nbv + c0 + kk] = (a0.x + a0.y) * scale;
+        sc[(2 * rp + 1) * nbv + c0 + kk] = (a1.x + a1.y) * scale;
+      }
     }
     __syncthreads();
   }
@@ -80,67 +172,59 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float* __restric
       if (lane == 0) cnt[bh * nb + i] = nb;
       continue;
     }
-    const float* srow = sc + r * nbv;
-    // k_eff-th largest key T: largest T with #{key >= T} >= k_eff.
-    uint32_t T = 0;
-    for (int b = 31; b >= 0; --b) {
-      const uint32_t cand = T | (1u << b);
-      int c = 0;
-      for (int j = lane; j < nbv; j += 32) c += (orderable_key(srow[j]) >= cand) ? 1 : 0;
-      c = __reduce_add_sync(0xffffffffu, c);
-      if (c >= k_eff) T = cand;
-    }
-    int gt = 0;
-    for (int j = lane; j < nbv; j += 32) gt += (orderable_key(srow[j]) > T) ? 1 : 0;
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    const int need_eq = k_eff - gt;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    int out = 0, eq_seen = 0;
-    for (int base = 0; base < nbv; base += 32) {
-      const int j = base + lane;
-      const uint32_t u = (j < nbv) ? orderable_key(srow[j]) : 0u;
-      const bool is_gt = (j < nbv) && (u > T);
-      const bool is_eq = (j < nbv) && (u == T);
-      const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
-      const bool sel = is_gt || (is_eq && (eq_seen + __popc(eqm & lt_mask)) < need_eq);
-      const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-      if (sel) row[pb + out + __popc(selm & lt_mask)] = pb + j;
-      out += __popc(selm);
-      eq_seen += __popc(eqm);
-    }
+    if (kPerLane > 0)
+      topk_row<(kPerLane > 0 ? kPerLane : 1)>(sc + r * nbv, nbv, k_eff, pb, row, lane);
+    else
+      topk_row_smem(sc + r * nbv, nbv, k_eff, pb, row, lane);
     for (int p = lane; p < pb; p += 32) row[p] = p;
     for (int p = pb + k_eff + lane; p < kcap; p += 32) row[p] = -1;
     if (lane == 0) cnt[bh * nb + i] = pb + k_eff;
   }
 }
 
-}  // namespace
-
-// Rows per CTA: up to 8, fewer when a row of scores is large, so the score
-// tile stays within 160 KB of shared memory.
-static int select_rows(int nbv) {
-  const int by_smem = (160 * 1024) / (nbv * 4 + kDim * 4);
-  return by_smem < 1 ? 1 : (by_smem > kMaxRows ? kMaxRows : by_smem);
-}
-
-cudaError_t launch_select(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
-                          int32_t* cnt, cudaStream_t st) {
-  const int R = select_rows(s.nbv);
-  const size_t smem = static_cast<size_t>(R) * (kDim + s.nbv) * sizeof(float);
+template <int kPerLane>
+cudaError_t launch_select_t(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
+                            int32_t* cnt, int R, size_t smem, cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         200 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(select_kernel<kPerLane>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   const dim3 grid((s.nb + R - 1) / R, s.B * s.H);
   const float scale = 0.088388347648318440550f;
-  select_kernel<<<grid, kThreads, smem, st>>>(qpool, kpool, idx, cnt, s.nb, s.pb, s.k_eff, s.kcap,
-                                              R, scale);
+  select_kernel<kPerLane><<<grid, kThreads, smem, st>>>(qpool, kpool, idx, cnt, s.nb, s.pb,
+                                                        s.k_eff, s.kcap, R, scale);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+// Query blocks per CTA: 16 (an even number, so the pair mapping covers it),
+// fewer when a row of scores is long, so the tile stays within ~180 KB.
+static int select_rows(int nbv) {
+  const size_t fixed = static_cast<size_t>(kChunk) * kPad * 4;
+  int R = 16;
+  while (R > 2 && fixed + static_cast<size_t>(R) * (kPad + nbv) * 4 > 180 * 1024) R -= 2;
+  return R;
+}
+
+cudaError_t launch_select(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
+                          int32_t* cnt, cudaStream_t st) {
+  const int R = select_rows(s.nbv);
+  const size_t smem = (static_cast<size_t>(R) * kPad + kChunk * kPad + static_cast<size_t>(R) * s.nbv) *
+                      sizeof(float);
+  // keys per lane: the smallest instantiation that holds the row
+  if (s.nbv <= 32 * 8) return launch_select_t<8>(s, qpool, kpool, idx, cnt, R, smem, st);
+  if (s.nbv <= 32 * 12) return launch_select_t<12>(s, qpool, kpool, idx, cnt, R, smem, st);
+  if (s.nbv <= 32 * 16) return launch_select_t<16>(s, qpool, kpool, idx, cnt, R, smem, st);
+  if (s.nbv <= 32 * 24) return launch_select_t<24>(s, qpool, kpool, idx, cnt, R, smem, st);
+  if (s.nbv <= 32 * 34) return launch_select_t<34>(s, qpool, kpool, idx, cnt, R, smem, st);
+  if (s.nbv <= 32 * 48) return launch_select_t<48>(s, qpool, kpool, idx, cnt, R, smem, st);
+  return launch_select_t<0>(s, qpool, kpool, idx, cnt, R, smem, st);
 }
 
 }  // namespace bsa

@@ -167,3 +167,11 @@ def test_density_sweep_sampled_head(rho):
     Q, K, V = _inputs(1, 2, N, cfg["kind"])
     buf = run_stages(Q, K, V, top_k, 0, "anchor", with_lse=False)
     check_head(buf, Q, K, V, 0, 1, top_k, 0, "anchor", check_lse=False)
+
+
+def test_long_rows_select_from_shared_memory():
+    # more than 1536 video blocks: the top-k keeps its keys in shared memory
+    N, top_k = 200_000, 8                       # 1563 blocks, ragged tail of 64 rows
+    Q, K, V = _inputs(1, 1, N, "block_offset", seed=21)
+    buf = run_stages(Q, K, V, top_k, 0, "anchor", with_lse=False)
+    check_head(buf, Q, K, V, 0, 0, top_k, 0, "anchor", check_lse=False)
