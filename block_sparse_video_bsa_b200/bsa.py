@@ -39,8 +39,19 @@ class bsa_params(ctypes.Structure):
     ]
 
 
+class bsa_fp8_operands(ctypes.Structure):
+    """Mirror of bsa_fp8_operands (include/bsa.h): e4m3 codes and fp32 scales."""
+    _fields_ = [("q8", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
+                ("k8", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
+                ("vt8", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
+                ("ks8", ctypes.c_void_p), ("ks_scale", ctypes.c_void_p),
+                ("vst8", ctypes.c_void_p), ("vs_scale", ctypes.c_void_p),
+                ("v_ref", ctypes.c_void_p)]
+
+
 _lib = None
 _P = ctypes.POINTER(bsa_params)
+_F8 = ctypes.POINTER(bsa_fp8_operands)
 _vp = ctypes.c_void_p
 _SIGS = {
     "bsa_num_blocks": (ctypes.c_int32, [_P]),
@@ -56,6 +67,12 @@ _SIGS = {
     "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_debug_expired_wait": (ctypes.c_int, [_vp, ctypes.c_uint64, _vp]),
     "bsa_forward_noalloc": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_fp8_operands_bytes": (ctypes.c_size_t, [_P]),
+    "bsa_fp8_operands_carve": (ctypes.c_int, [_P, _vp, ctypes.c_size_t, _F8]),
+    "bsa_quantize_fp8": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _F8, _vp]),
+    "bsa_attend_fp8": (ctypes.c_int, [_P, _F8, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_forward_fp8_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "bsa_forward_fp8": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
 }
 
 
@@ -164,6 +181,38 @@ def bsa_forward_noalloc(p, Q, K, V, O, lse=None, stream=None):
                                      _ptr(lse), _stream(stream)), "bsa_forward_noalloc")
 
 
+def bsa_fp8_operands_bytes(p: bsa_params) -> int:
+    return lib().bsa_fp8_operands_bytes(ctypes.byref(p))
+
+
+def bsa_fp8_operands_carve(p, buf) -> bsa_fp8_operands:
+    ops = bsa_fp8_operands()
+    _check(lib().bsa_fp8_operands_carve(ctypes.byref(p), _ptr(buf), buf.numel() * buf.element_size(),
+                                        ctypes.byref(ops)), "bsa_fp8_operands_carve")
+    return ops
+
+
+def bsa_quantize_fp8(p, Q, K, V, ksum, vsum, ops, stream=None):
+    _check(lib().bsa_quantize_fp8(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(ksum),
+                                  _ptr(vsum), ctypes.byref(ops), _stream(stream)),
+           "bsa_quantize_fp8")
+
+
+def bsa_attend_fp8(p, ops, idx, cnt, bias, O, lse=None, stream=None):
+    _check(lib().bsa_attend_fp8(ctypes.byref(p), ctypes.byref(ops), _ptr(idx), _ptr(cnt),
+                                _ptr(bias), _ptr(O), _ptr(lse), _stream(stream)), "bsa_attend_fp8")
+
+
+def bsa_forward_fp8_workspace_bytes(p: bsa_params) -> int:
+    return lib().bsa_forward_fp8_workspace_bytes(ctypes.byref(p))
+
+
+def bsa_forward_fp8(p, Q, K, V, O, lse, workspace, stream=None):
+    _check(lib().bsa_forward_fp8(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream)), "bsa_forward_fp8")
+
+
 def bsa_debug_expired_wait(dev_status, timeout_ns: int, stream=None):
     _check(lib().bsa_debug_expired_wait(_ptr(dev_status), int(timeout_ns), _stream(stream)),
            "bsa_debug_expired_wait")
@@ -207,6 +256,48 @@ def forward(Q, K, V, top_k, prefix=0, variant="anchor", return_lse=False, ws=Non
     if ws is None:
         ws = workspace(p, Q.device)
     bsa_forward(p, Q, K, V, O, lse, ws, stream)
+    return (O, lse) if return_lse else O
+
+
+def fp8_operands(p: bsa_params, device="cuda"):
+    """One FP8 operand set in a fresh device buffer: (buffer, struct, views).
+
+    ``views`` maps each field of bsa_fp8_operands to a torch view of the
+    buffer with the documented shape (codes as uint8)."""
+    n = bsa_fp8_operands_bytes(p)
+    if n == 0:
+        raise BsaError(BSA_ERR_INVALID, "bsa_fp8_operands_bytes")
+    buf = torch.empty(n, dtype=torch.uint8, device=device)
+    ops = bsa_fp8_operands_carve(p, buf)
+    B, H, N = p.B, p.H, p.N
+    nb = bsa_num_blocks(p)
+    nt = -(-nb // 128)
+    shapes = dict(q8=(B, H, N, 128), q_scale=(B, H, nb), k8=(B, H, N, 128), k_scale=(B, H, nb),
+                  vt8=(B, H, nb, 128, 128), v_scale=(B, H, nb), ks8=(B, H, nb, 128),
+                  ks_scale=(B, H, nt), vst8=(B, H, nt, 128, 128), vs_scale=(B, H, nt),
+                  v_ref=(B, H))
+    base = buf.data_ptr()
+    views = {}
+    for name, shape in shapes.items():
+        off = getattr(ops, name) - base
+        count = math.prod(shape)
+        if name.endswith("8"):
+            views[name] = buf[off:off + count].view(shape)
+        else:
+            views[name] = buf[off:off + 4 * count].view(torch.float32).view(shape)
+    return buf, ops, views
+
+
+def forward_fp8(Q, K, V, top_k, prefix=0, variant="anchor", return_lse=False, ws=None,
+                stream=None):
+    """bsa_forward_fp8: the same call as ``forward`` with e4m3 attention operands."""
+    B, H, N, D = Q.shape
+    p = params(B, H, N, top_k, prefix, variant, D=D)
+    O = torch.empty_like(Q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=Q.device) if return_lse else None
+    if ws is None:
+        ws = torch.empty(bsa_forward_fp8_workspace_bytes(p), dtype=torch.uint8, device=Q.device)
+    bsa_forward_fp8(p, Q, K, V, O, lse, ws, stream)
     return (O, lse) if return_lse else O
 
 

@@ -17,7 +17,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbsa.so")
 BUILD_DIR = os.path.join(PKG, "_build")
-SOURCES = ["api.cu", "pool_summarize.cu", "select.cu", "attend.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "pool_summarize.cu", "select.cu", "attend.cu", "attend_fp8.cu", "quant_fp8.cu",
+           "noalloc.cu"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

@@ -93,7 +93,79 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t BH) {
          CUDA_SUCCESS;
 }
 
+// uint8 (e4m3 codes) [BH, rows, 128] viewed as a 3-D tensor; box = 128
+// columns (128 bytes, one swizzle atom) x 128 rows x 1 head.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {128, rows, BH};
+  const cuuint64_t strides[2] = {128, rows * 128};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// The FP8 operand set carved from one buffer in the order of
+// bsa_fp8_operands (each piece 256-byte aligned); returns the bytes used.
+size_t fp8_carve(const Shape& s, uint8_t* base, bsa::Fp8Operands* f) {
+  const size_t bh = static_cast<size_t>(s.B) * s.H;
+  const size_t ntile = (s.nb + 127) / 128;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += round256(bytes);
+    return p;
+  };
+  uint8_t* q8 = take(bh * s.N * 128);
+  uint8_t* qs = take(bh * s.nb * 4);
+  uint8_t* k8 = take(bh * s.N * 128);
+  uint8_t* ks = take(bh * s.nb * 4);
+  uint8_t* vt8 = take(bh * s.nb * 128 * 128);
+  uint8_t* vs = take(bh * s.nb * 4);
+  uint8_t* ks8 = take(bh * s.nb * 128);
+  uint8_t* kss = take(bh * ntile * 4);
+  uint8_t* vst8 = take(bh * ntile * 128 * 128);
+  uint8_t* vss = take(bh * ntile * 4);
+  uint8_t* vref = take(bh * 4);
+  if (f) {
+    f->q8 = q8;
+    f->q_scale = reinterpret_cast<float*>(qs);
+    f->k8 = k8;
+    f->k_scale = reinterpret_cast<float*>(ks);
+    f->vt8 = vt8;
+    f->v_scale = reinterpret_cast<float*>(vs);
+    f->ks8 = ks8;
+    f->ks_scale = reinterpret_cast<float*>(kss);
+    f->vst8 = vst8;
+    f->vs_scale = reinterpret_cast<float*>(vss);
+    f->v_ref = reinterpret_cast<float*>(vref);
+  }
+  return off;
+}
+
+bsa::Fp8Operands from_abi(const bsa_fp8_operands& o) {
+  return bsa::Fp8Operands{o.q8, o.q_scale, o.k8, o.k_scale, o.vt8, o.v_scale,
+                          o.ks8, o.ks_scale, o.vst8, o.vs_scale, o.v_ref};
+}
+
+bool fp8_valid(const bsa_fp8_operands* o) {
+  if (!o || !o->q8 || !o->q_scale || !o->k8 || !o->k_scale || !o->vt8 || !o->v_scale ||
+      !o->ks8 || !o->ks_scale || !o->vst8 || !o->vs_scale || !o->v_ref)
+    return false;
+  return true;
+}
+
+bool fp8_aligned(const bsa_fp8_operands* o) {
+  return aligned(o->q8, 16) && aligned(o->k8, 16) && aligned(o->vt8, 16) && aligned(o->ks8, 16) &&
+         aligned(o->vst8, 16) && aligned(o->q_scale, 4) && aligned(o->k_scale, 4) &&
+         aligned(o->v_scale, 4) && aligned(o->ks_scale, 4) && aligned(o->vs_scale, 4) &&
+         aligned(o->v_ref, 4);
+}
 
 struct Workspace {
   float *qpool, *anchor, *kpool, *bias;
@@ -156,9 +228,105 @@ int attend_impl(const Shape& s, const void* Q, const void* K, const void* V, con
   return cuda_status(bsa::launch_attend(s, maps, idx, cnt, bias, O, lse, st));
 }
 
+int quantize_fp8_impl(const Shape& s, const void* Q, const void* K, const void* V,
+                      const void* ksum, const void* vsum, const bsa::Fp8Operands& f,
+                      cudaStream_t st) {
+  return cuda_status(bsa::launch_quantize_fp8(s, Q, K, V, ksum, vsum, f, st));
+}
+
+int attend_fp8_impl(const Shape& s, const bsa::Fp8Operands& f, const int32_t* idx,
+                    const float* bias, void* O, float* lse, cudaStream_t st) {
+  bsa::AttendMapsFp8 maps;
+  const uint64_t bh = static_cast<uint64_t>(s.B) * s.H;
+  const uint64_t ntile = (s.nb + 127) / 128;
+  if (!make_map_u8(&maps.q, f.q8, s.N, bh) || !make_map_u8(&maps.k, f.k8, s.N, bh) ||
+      !make_map_u8(&maps.vt, f.vt8, static_cast<uint64_t>(s.nb) * 128, bh) ||
+      !make_map_u8(&maps.ks, f.ks8, s.nb, bh) ||
+      !make_map_u8(&maps.vst, f.vst8, ntile * 128, bh))
+    return BSA_ERR_UNSUPPORTED;
+  return cuda_status(bsa::launch_attend_fp8(s, maps, f, idx, bias, O, lse, st));
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t bsa_fp8_operands_bytes(const bsa_params* p) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK) return 0;
+  return fp8_carve(s, nullptr, nullptr);
+}
+
+int bsa_fp8_operands_carve(const bsa_params* p, void* base, size_t bytes, bsa_fp8_operands* out) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!base || !out || bytes < fp8_carve(s, nullptr, nullptr)) return BSA_ERR_INVALID;
+  if (!aligned(base, 256)) return BSA_ERR_ALIGN;
+  bsa::Fp8Operands f;
+  fp8_carve(s, static_cast<uint8_t*>(base), &f);
+  *out = bsa_fp8_operands{f.q8, f.q_scale, f.k8, f.k_scale, f.vt8, f.v_scale,
+                          f.ks8, f.ks_scale, f.vst8, f.vs_scale, f.v_ref};
+  return BSA_OK;
+}
+
+int bsa_quantize_fp8(const bsa_params* p, const void* Q, const void* K, const void* V,
+                     const void* ksum, const void* vsum, const bsa_fp8_operands* ops,
+                     void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !K || !V || !ksum || !vsum || !fp8_valid(ops)) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(ksum, 16) ||
+      !aligned(vsum, 16) || !fp8_aligned(ops))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return quantize_fp8_impl(s, Q, K, V, ksum, vsum, from_abi(*ops),
+                           static_cast<cudaStream_t>(stream));
+}
+
+int bsa_attend_fp8(const bsa_params* p, const bsa_fp8_operands* ops, const int32_t* idx,
+                   const int32_t* cnt, const float* bias, void* O, float* lse, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!fp8_valid(ops) || !idx || !cnt || !bias || !O) return BSA_ERR_INVALID;
+  if (!fp8_aligned(ops) || !aligned(O, 16) || !aligned(idx, 4) || !aligned(cnt, 4) ||
+      !aligned(bias, 4) || (lse && !aligned(lse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return attend_fp8_impl(s, from_abi(*ops), idx, bias, O, lse, static_cast<cudaStream_t>(stream));
+}
+
+size_t bsa_forward_fp8_workspace_bytes(const bsa_params* p) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK) return 0;
+  return carve(s, nullptr, nullptr) + fp8_carve(s, nullptr, nullptr);
+}
+
+int bsa_forward_fp8(const bsa_params* p, const void* Q, const void* K, const void* V, void* O,
+                    float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !workspace) return BSA_ERR_INVALID;
+  const size_t ws0 = carve(s, nullptr, nullptr);
+  if (workspace_bytes < ws0 + fp8_carve(s, nullptr, nullptr)) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
+      !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  Workspace w;
+  carve(s, static_cast<uint8_t*>(workspace), &w);
+  bsa::Fp8Operands f;
+  fp8_carve(s, static_cast<uint8_t*>(workspace) + ws0, &f);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = pool_impl(s, Q, w.qpool, w.anchor, st))) return rc;
+  if ((rc = summarize_impl(s, K, V, w.anchor, w.kpool, w.ksum, w.vsum, w.bias, st))) return rc;
+  if ((rc = select_impl(s, w.qpool, w.kpool, w.idx, w.cnt, st))) return rc;
+  if ((rc = quantize_fp8_impl(s, Q, K, V, w.ksum, w.vsum, f, st))) return rc;
+  return attend_fp8_impl(s, f, w.idx, w.bias, O, lse, st);
+}
 
 int32_t bsa_num_blocks(const bsa_params* p) {
   Shape s;

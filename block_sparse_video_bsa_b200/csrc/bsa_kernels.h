@@ -32,6 +32,33 @@ struct AttendMaps {
 cudaError_t launch_attend(const Shape& s, const AttendMaps& maps, const int32_t* idx,
                           const int32_t* cnt, const float* bias, void* O, float* lse,
                           cudaStream_t st);
+// FP8 (e4m3) operands (layouts as bsa_fp8_operands in include/bsa.h).
+struct Fp8Operands {
+  void* q8;
+  float* q_scale;
+  void* k8;
+  float* k_scale;
+  void* vt8;
+  float* v_scale;
+  void* ks8;
+  float* ks_scale;
+  void* vst8;
+  float* vs_scale;
+  float* v_ref;
+};
+cudaError_t launch_quantize_fp8(const Shape& s, const void* Q, const void* K, const void* V,
+                                const void* ksum, const void* vsum, const Fp8Operands& f,
+                                cudaStream_t st);
+
+struct AttendMapsFp8 {
+  // uint8, box {128, 128, 1}, 128B swizzle: q8, k8 [BH, N, 128]; vt8
+  // [BH, nb * 128, 128]; ks8 [BH, nb, 128]; vst8 [BH, ntile * 128, 128]
+  CUtensorMap q, k, vt, ks, vst;
+};
+cudaError_t launch_attend_fp8(const Shape& s, const AttendMapsFp8& maps, const Fp8Operands& f,
+                              const int32_t* idx, const float* bias, void* O, float* lse,
+                              cudaStream_t st);
+
 cudaError_t launch_expired_wait(int32_t* dev_status, uint64_t timeout_ns, cudaStream_t st);
 
 }  // namespace bsa

@@ -190,6 +190,75 @@ int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK,
 int bsa_forward_noalloc(const bsa_params* p, const void* Q, const void* K, const void* V,
                         void* O, float* lse, void* stream);
 
+/* ---- FP8 (e4m3) exact and compressed branch --------------------------- */
+
+/* The pages name a quantised sparse kernel ("H3 Sparse Attention", comfy.icu
+ * WAS node, section "What it actually does": the sparse layers compute in
+ * INT8 inside the kernel, at some cost in fidelity).  This is that option
+ * with FP8: the attention operands are e4m3 codes, the path before it (pool,
+ * summarize, select) is the bf16 path unchanged.  Format and scaling are this
+ * library's reading:
+ *   - e4m3 (OCP FP8, max 448), round to nearest even, saturating;
+ *   - one scale per 128-row group: each 128-token block of Q, K and V (real
+ *     rows only) and each 128-row tile of the summary tables k~ and v~;
+ *   - codes = e4m3(x * fp32(448 / amax)), scale = fp32(amax / 448) (both 1
+ *     for an all-zero group);
+ *   - in the kernel, logits use the scales of the query block and of the key
+ *     block / summary tile; softmax numerators p enter the PV product as
+ *     e4m3(p * s_v / v_ref), v_ref the head's largest value scale, and the
+ *     row sum stays in fp32.
+ * All pointers are device pointers owned by the caller (16-byte aligned for
+ * the code arrays, 4-byte for the scales).  ntile = ceil(nb / 128). */
+typedef struct {
+  void* q8;         /* e4m3 [B,H,N,128], row-major like Q                     */
+  float* q_scale;   /* [B,H,nb]                                               */
+  void* k8;         /* e4m3 [B,H,N,128]                                       */
+  float* k_scale;   /* [B,H,nb]                                               */
+  void* vt8;        /* e4m3 [B,H,nb,128,128]: block j of V as [dim][key],
+                       keys past N zero                                       */
+  float* v_scale;   /* [B,H,nb]                                               */
+  void* ks8;        /* e4m3 [B,H,nb,128], the bf16 k~ rows quantised per tile */
+  float* ks_scale;  /* [B,H,ntile]                                            */
+  void* vst8;       /* e4m3 [B,H,ntile,128,128]: tile u of v~ as [dim][row],
+                       rows past nb zero                                      */
+  float* vs_scale;  /* [B,H,ntile]                                            */
+  float* v_ref;     /* [B,H]: max of v_scale and vs_scale of the head         */
+} bsa_fp8_operands;
+
+/* Bytes of one operand set carved from a single buffer (each piece 256-byte
+ * aligned, in field order); 0 for invalid parameters. */
+size_t bsa_fp8_operands_bytes(const bsa_params* p);
+
+/* Fills *out with pointers into the caller's buffer `base` (256-byte
+ * aligned, at least bsa_fp8_operands_bytes(p) bytes).  Allocates nothing. */
+int bsa_fp8_operands_carve(const bsa_params* p, void* base, size_t bytes,
+                           bsa_fp8_operands* out);
+
+/* Quantises Q, K, V (bf16 [B,H,N,128]) and the summary tables ksum, vsum
+ * (bf16 [B,H,nb,128] as bsa_summarize wrote them) into *ops, and writes
+ * ops->v_ref.  Six launches on `stream`; every byte of *ops is written. */
+int bsa_quantize_fp8(const bsa_params* p, const void* Q, const void* K, const void* V,
+                     const void* ksum, const void* vsum, const bsa_fp8_operands* ops,
+                     void* stream);
+
+/* bsa_attend on the e4m3 operands of bsa_quantize_fp8 (tcgen05
+ * kind::f8f6f4, fp32 accumulate in TMEM), with the same idx/cnt/bias and the
+ * same outputs (O bf16, optional lse). */
+int bsa_attend_fp8(const bsa_params* p, const bsa_fp8_operands* ops, const int32_t* idx,
+                   const int32_t* cnt, const float* bias, void* O, float* lse,
+                   void* stream);
+
+/* Workspace of bsa_forward_fp8: bsa_workspace_bytes(p) followed by one
+ * operand set. */
+size_t bsa_forward_fp8_workspace_bytes(const bsa_params* p);
+
+/* bsa_pool, bsa_summarize, bsa_select, bsa_quantize_fp8, bsa_attend_fp8 in
+ * order on `stream`, intermediates in the caller's workspace (256-byte
+ * aligned, at least bsa_forward_fp8_workspace_bytes(p) bytes). */
+int bsa_forward_fp8(const bsa_params* p, const void* Q, const void* K, const void* V,
+                    void* O, float* lse, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
 /* Human-readable name of a bsa_status value (static string). */
 const char* bsa_status_string(int status);
 

@@ -134,7 +134,7 @@ def forward_head_fp8(Q, K, V, top_k: int, prefix: int = 0, variant: str = "ancho
 
 
 def fp8_output_bound(Qd, Kd, Vd, lists, KSd, VSd, bias, v_scale, vs_scale, prefix_blocks: int,
-                     block: int = BLOCK, query_blocks=None):
+                     block: int = BLOCK, query_blocks=None, with_variance: bool = False):
     """Per-element bound on |O_kernel - O| from the kernel's e4m3 numerators.
 
     The kernel writes each softmax numerator p (relative to a running max at
@@ -145,6 +145,12 @@ def fp8_output_bound(Qd, Kd, Vd, lists, KSd, VSd, bias, v_scale, vs_scale, prefi
     column's weight moves by at most max(2^-4 w, 2^-10 / (r * l)), with w the
     exact weight and l = sum_t exp(x_t - max) the exact row sum.  The bound is
     the sum of those moves times |v|, column by column.
+
+    With ``with_variance`` it also returns an upper model of each element's
+    error variance: rounding to nearest leaves an error spread over at most
+    half a step, so a move of at most m has variance at most m^2 / 3 (the
+    uniform case); the moves of different columns are independent roundings,
+    so the variances add: sum_t max-move_t^2 / 3 * v_t^2.
     """
     Qd = np.asarray(Qd, dtype=np.float64)
     N, d = Qd.shape
@@ -154,6 +160,7 @@ def fp8_output_bound(Qd, Kd, Vd, lists, KSd, VSd, bias, v_scale, vs_scale, prefi
     pb = prefix_blocks
     s_ref = max(np.max(v_scale), np.max(vs_scale))
     out = np.zeros((N, d))
+    var = np.zeros((N, d))
     for i, (a, b) in enumerate(bounds):
         if query_blocks is not None and i not in query_blocks:
             continue
@@ -174,4 +181,5 @@ def fp8_output_bound(Qd, Kd, Vd, lists, KSd, VSd, bias, v_scale, vs_scale, prefi
         l = p.sum(axis=1, keepdims=True)
         move = np.maximum(2.0 ** -4 * p / l, 2.0 ** -10 / (r[None, :] * l))
         out[a:b] = move @ vals
-    return out
+        var[a:b] = (move ** 2 / 3) @ (vals ** 2)
+    return (out, var) if with_variance else out

@@ -129,8 +129,10 @@ def test_output_bound_covers_simulated_e4m3_numerators():
     K = rng.standard_normal((N, d)) * 1.5
     V = rng.standard_normal((N, d))
     r8 = f8.forward_head_fp8(Q, K, V, top_k, 0)
-    bound = f8.fp8_output_bound(r8["Qd"], r8["Kd"], r8["Vd"], r8["lists"], r8["KSd"], r8["VSd"],
-                                r8["bias"], r8["v_scale"], r8["vs_scale"], 0)
+    bound, var = f8.fp8_output_bound(r8["Qd"], r8["Kd"], r8["Vd"], r8["lists"], r8["KSd"],
+                                     r8["VSd"], r8["bias"], r8["v_scale"], r8["vs_scale"], 0,
+                                     with_variance=True)
+    sq_err = 0.0
     s_ref = max(r8["v_scale"].max(), r8["vs_scale"].max())
     bounds = orc.block_bounds(N)
     nb = len(bounds)
@@ -149,3 +151,6 @@ def test_output_bound_covers_simulated_e4m3_numerators():
         err = np.abs(O_sim - r8["O"][a:b])
         assert (err <= bound[a:b] + 1e-12).all()
         assert err.max() > 0
+        sq_err += float((err ** 2).sum())
+    # the squared error over all elements stays within the variance model
+    assert sq_err <= var.sum(), (sq_err, var.sum())
