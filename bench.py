@@ -2,10 +2,15 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload h3_768p_5s] [--top-k K] [--no-cpu-baseline] [--no-e2e]
+                    [--precision bf16|fp8]
 
 One step = one whole attention call (pool -> summarize -> select -> attend,
 all through the C ABI) over one batch of synthetic bf16 input of the 768p-5s
 H3 shape (B=1, H=56, N=37,740, d=128, top_k=64, anchor-weighted summaries).
+``--precision fp8`` times the FP8 (e4m3) option instead: the same stages plus
+the quantisation of the attention operands, then the e4m3 attention kernel;
+its roofline peak is the measured bf16 peak times the nominal e4m3/bf16
+tensor ratio (2).  The default (bf16) line is the headline.
 Prints ONE JSON line on rank 0.  Multi-GPU (torchrun): every rank runs its own
 independent call on its own inputs (weak scaling, no data-path collective);
 the time is the max over ranks.
@@ -45,6 +50,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"])
     return ap.parse_args()
 
 
@@ -172,9 +178,12 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle
 
-def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3):
-    """The fp64 oracle as it stands, on whole heads, until ~budget_s of CPU work."""
+def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False):
+    """The fp64 oracle as it stands, on whole heads, until ~budget_s of CPU work
+    (the FP8 oracle for ``fp8``)."""
     import oracle as orc
+    from oracle import bsa_oracle_fp8 as orc8
+    head_fn = orc8.forward_head_fp8 if fp8 else orc.forward_head
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
@@ -184,7 +193,7 @@ def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3):
     t0 = time.perf_counter()
     heads = 0
     for h in range(min(max_heads, len(Qh))):
-        out = orc.forward_head(Qh[h], Kh[h], Vh[h], cfg["top_k"], cfg["prefix"], cfg["variant"])
+        out = head_fn(Qh[h], Kh[h], Vh[h], cfg["top_k"], cfg["prefix"], cfg["variant"])
         pairs += orc.effective_pairs(len(Qh[h]), out["lists"], cfg["prefix"] // 128)
         heads += 1
         if time.perf_counter() - t0 > budget_s:
@@ -192,7 +201,8 @@ def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3):
     dt = time.perf_counter() - t0
     flops = 4 * 128 * pairs
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{heads} of {cfg['H']} heads of the workload, whole path per head "
+            "sample": f"{heads} of {cfg['H']} heads of the workload, whole "
+                      f"{'FP8 ' if fp8 else ''}path per head "
                       f"(numpy fp64, BLAS threads = {cores}); {dt:.1f} s, "
                       f"{dt / heads:.2f} s/head"}, dt / heads
 
@@ -292,24 +302,34 @@ def main():
     buf = bsa.stage_buffers(B, H, N, top_k, prefix, variant, device=dev)
     O = torch.empty_like(Q)
     stream = torch.cuda.current_stream(dev)
+    fp8 = args.precision == "fp8"
+    if fp8:
+        ops_buf, ops, _ = bsa.fp8_operands(p, dev)
+    names = ["pool", "summarize", "select"] + (["quantize"] if fp8 else []) + ["attend"]
+    nev = len(names) + 1
 
     def step(ev=None):
-        if ev:
-            ev[0].record(stream)
+        marks = iter(ev or [])
+
+        def mark():
+            if ev:
+                next(marks).record(stream)
+        mark()
         bsa.bsa_pool(p, Q, buf["qpool"], buf["anchor"], stream)
-        if ev:
-            ev[1].record(stream)
+        mark()
         bsa.bsa_summarize(p, K, V, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"],
                           buf["bias"], stream)
-        if ev:
-            ev[2].record(stream)
+        mark()
         bsa.bsa_select(p, buf["qpool"], buf["kpool"], buf["idx"], buf["cnt"], stream)
-        if ev:
-            ev[3].record(stream)
-        bsa.bsa_attend(p, Q, K, V, buf["idx"], buf["cnt"], buf["ksum"], buf["vsum"], buf["bias"],
-                       O, None, stream)
-        if ev:
-            ev[4].record(stream)
+        mark()
+        if fp8:
+            bsa.bsa_quantize_fp8(p, Q, K, V, buf["ksum"], buf["vsum"], ops, stream)
+            mark()
+            bsa.bsa_attend_fp8(p, ops, buf["idx"], buf["cnt"], buf["bias"], O, None, stream)
+        else:
+            bsa.bsa_attend(p, Q, K, V, buf["idx"], buf["cnt"], buf["ksum"], buf["vsum"],
+                           buf["bias"], O, None, stream)
+        mark()
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -321,7 +341,8 @@ def main():
     flops_step = 4 * 128 * pairs
     nb = bsa.bsa_num_blocks(p)
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+              for _ in range(args.steps)]
     clocks = ClockSampler(local)
     if world > 1:
         dist.barrier()
@@ -337,15 +358,47 @@ def main():
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {bsa.status_string(int(status.item()))}")
 
-    total_ms = sum(e[0].elapsed_time(e[4]) for e in events)
-    stage_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in events) for i in range(4)]
+    total_ms = sum(e[0].elapsed_time(e[-1]) for e in events)
+    stage_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in events)
+                for i in range(nev - 1)]
     total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
     value = job_tflops(flops_step, args.steps, world, total_ms)
 
     # end to end through the C ABI from pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and fp8:
+        # the public FP8 call from pinned host buffers: copies in, forward_fp8,
+        # O copied back, all inside the timed region
+        hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
+        hO = torch.empty_like(hQ).pin_memory()
+        ws8 = torch.empty(bsa.bsa_forward_fp8_workspace_bytes(p), dtype=torch.uint8, device=dev)
+
+        def e2e_call():
+            Q.copy_(hQ, non_blocking=True)
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            bsa.bsa_forward_fp8(p, Q, K, V, O, None, ws8, stream)
+            hO.copy_(O, non_blocking=True)
+        for _ in range(2):
+            e2e_call()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_call()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": job_tflops(flops_step, args.e2e_steps, world, e_ms),
+               "unit": "TFLOP/s", "ms_per_call": e_ms / args.e2e_steps,
+               "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
+               "d2h_bytes_per_step": O.numel() * O.element_size(),
+               "path": "bsa_forward_fp8 with pinned-host copies in and out (one stream)"}
+        del hQ, hK, hV, hO, ws8
+    elif not args.no_e2e:
         hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
         hO = torch.empty_like(hQ).pin_memory()
         ws = bsa.workspace(p, dev)
@@ -369,9 +422,9 @@ def main():
         del hQ, hK, hV, hO
 
     peaks, peak_src = load_peaks()
-    attend_ms = stage_ms[3]
+    attend_ms = stage_ms[-1]
     attend_tflops = flops_step / (attend_ms / 1e3) / 1e12
-    peak = float(peaks["bf16_tflops"])
+    peak = float(peaks["bf16_tflops"]) * (2.0 if fp8 else 1.0)
     pool_bytes = stage_bytes(B, H, N, nb, bsa.bsa_select_capacity(p))
     pool_gbs = pool_bytes / ((stage_ms[0] + stage_ms[1]) / 1e3) / 1e9
 
@@ -381,30 +434,32 @@ def main():
         Qh = [Q[0, h].double().cpu().numpy() for h in hh]
         Kh = [K[0, h].double().cpu().numpy() for h in hh]
         Vh = [V[0, h].double().cpu().numpy() for h in hh]
-        cpu, _ = time_oracle(Qh, Kh, Vh, cfg)
+        cpu, _ = time_oracle(Qh, Kh, Vh, cfg, fp8=fp8)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if fp8 else "bf16",
             "data": "synthetic (seeded per-block-offset bf16 Q/K/V of the H3 768p-5s shape)",
             "config": config_block(cfg, parallelism=f"{world} independent calls (one per GPU)"),
             "ms_per_call": ms_per_step,
             "effective_tflop_per_call": flops_step / 1e12,
-            "stages_ms": {"pool": stage_ms[0], "summarize": stage_ms[1], "select": stage_ms[2],
-                          "attend": stage_ms[3]},
-            "roofline": {"kernel": "attend_kernel", "bound": "tensor", "achieved": attend_tflops,
+            "stages_ms": dict(zip(names, stage_ms)),
+            "roofline": {"kernel": "attend_fp8_kernel" if fp8 else "attend_kernel",
+                         "bound": "tensor", "achieved": attend_tflops,
                          "peak": peak, "unit": "TFLOP/s", "frac": attend_tflops / peak,
-                         "peak_source": f"{peak_src} bf16 burst",
-                         "traffic": read_traffic(cfg)},
+                         "peak_source": f"{peak_src} bf16 burst"
+                                        + (" x 2 (nominal e4m3/bf16 ratio)" if fp8 else ""),
+                         "traffic": read_traffic(cfg, "attend_fp8" if fp8 else "attend")},
             "pool_summary": {"bound": "hbm", "achieved": pool_gbs,
                              "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                              "frac": pool_gbs / float(peaks["hbm_gbs"]),
                              "bytes_per_call": pool_bytes},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": (11 if fp8 else 5) * args.steps,
             "clocks": clock_info,
             "context": {"pages_rtx_pro_6000_sparse_ms": 30.7 if cfg["N"] == 37_740 else None},
         }
@@ -414,11 +469,12 @@ def main():
         dist.destroy_process_group()
 
 
-def read_traffic(cfg):
-    """DRAM bytes per attend launch from the committed ncu summary, if it was
+def read_traffic(cfg, kernel="attend"):
+    """DRAM bytes per launch of the attention kernel (source csrc/<kernel>.cu)
+    from the committed ncu summary profiles/<kernel>_traffic.txt, if it was
     taken on the current kernel source and this workload; else None."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "attend_traffic.txt")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
     if not os.path.exists(path):
         return None
     kv = {}
@@ -426,9 +482,9 @@ def read_traffic(cfg):
         if "=" in ln and not ln.startswith("#"):
             k, v = ln.split("=", 1)
             kv[k.strip()] = v.strip()
-    src = os.path.join(ROOT, "block_sparse_video_bsa_b200", "csrc", "attend.cu")
+    src = os.path.join(ROOT, "block_sparse_video_bsa_b200", "csrc", f"{kernel}.cu")
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if kv.get("attend_cu_sha256_16") != h or kv.get("workload") != cfg["name"]:
+    if kv.get(f"{kernel}_cu_sha256_16") != h or kv.get("workload") != cfg["name"]:
         return None
     try:
         return float(kv["dram_bytes_per_launch"])
