@@ -134,17 +134,23 @@ def test_fp8_forward_matches_stages_and_is_deterministic():
     assert torch.equal(l1, buf["lse"]) and torch.equal(l1, l2)
 
 
-def test_fp8_full_size_sampled_head():
-    # the 768p-5s workload through bsa_forward_fp8 (the call bench.py times
-    # with --precision fp8); one head against the oracle on 24 query blocks
-    cfg = CONFIGS["h3_768p_5s"]
+@pytest.mark.parametrize("name,head,n_qb", [("h3_768p_5s", 31, 24),
+                                            ("h3_768p_15s_prefix512", 5, 12),
+                                            ("h3_2k_5s", 17, 8)])
+def test_fp8_full_size_sampled_head(name, head, n_qb):
+    # the workload through bsa_forward_fp8 (the call bench.py times with
+    # --precision fp8); one head against the oracle on sampled query blocks
+    # (the prefix workload's sample includes two dense-prefix query blocks)
+    cfg = CONFIGS[name]
     B, H, N = cfg["B"], cfg["H"], cfg["N"]
     Q, K, V = make_qkv(B, H, N, 128, cfg["kind"], 0, device="cuda")
     O = bsa.forward_fp8(Q, K, V, cfg["top_k"], cfg["prefix"], cfg["variant"])
     buf = run_fp8_stages(Q, K, V, cfg["top_k"], cfg["prefix"], cfg["variant"], with_lse=False)
     assert torch.equal(O, buf["O"])
-    qb = sorted(np.random.default_rng(7).choice(-(-N // 128), 24, replace=False).tolist())
-    check_head_fp8(buf, Q, K, V, 0, 31, cfg["top_k"], cfg["prefix"], cfg["variant"],
-                   check_lse=False, query_blocks=qb)
+    qb = set(np.random.default_rng(7).choice(-(-N // 128), n_qb, replace=False).tolist())
+    if cfg["prefix"]:
+        qb |= {0, cfg["prefix"] // 128 - 1}
+    check_head_fp8(buf, Q, K, V, 0, head, cfg["top_k"], cfg["prefix"], cfg["variant"],
+                   check_lse=False, query_blocks=sorted(qb))
     del Q, K, V, O, buf
     torch.cuda.empty_cache()
