@@ -67,6 +67,13 @@ _SIGS = {
     "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_debug_expired_wait": (ctypes.c_int, [_vp, ctypes.c_uint64, _vp]),
     "bsa_forward_noalloc": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_reblock_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "bsa_reblock": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "bsa_permute": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_unpermute": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_forward_reblock_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "bsa_forward_reblock": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                           _vp]),
     "bsa_fp8_operands_bytes": (ctypes.c_size_t, [_P]),
     "bsa_fp8_operands_carve": (ctypes.c_int, [_P, _vp, ctypes.c_size_t, _F8]),
     "bsa_quantize_fp8": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _F8, _vp]),
@@ -179,6 +186,62 @@ def bsa_forward_noalloc(p, Q, K, V, O, lse=None, stream=None):
     for callers that cannot allocate device memory (see include/bsa.h)."""
     _check(lib().bsa_forward_noalloc(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
                                      _ptr(lse), _stream(stream)), "bsa_forward_noalloc")
+
+
+def bsa_reblock_workspace_bytes(p: bsa_params) -> int:
+    return lib().bsa_reblock_workspace_bytes(ctypes.byref(p))
+
+
+def bsa_reblock(p, Q, K, perm, workspace, stream=None):
+    _check(lib().bsa_reblock(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(perm), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)),
+           "bsa_reblock")
+
+
+def bsa_permute(p, Q, K, V, perm, Qp, Kp, Vp, stream=None):
+    _check(lib().bsa_permute(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(Qp),
+                             _ptr(Kp), _ptr(Vp), _stream(stream)), "bsa_permute")
+
+
+def bsa_unpermute(p, Op, lsep, perm, O, lse=None, stream=None):
+    _check(lib().bsa_unpermute(ctypes.byref(p), _ptr(Op), _ptr(lsep), _ptr(perm), _ptr(O),
+                               _ptr(lse), _stream(stream)), "bsa_unpermute")
+
+
+def bsa_forward_reblock_workspace_bytes(p: bsa_params) -> int:
+    return lib().bsa_forward_reblock_workspace_bytes(ctypes.byref(p))
+
+
+def bsa_forward_reblock(p, Q, K, V, O, lse, workspace, stream=None):
+    _check(lib().bsa_forward_reblock(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                     _ptr(lse), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream(stream)), "bsa_forward_reblock")
+
+
+def reblock(Q, K, prefix=0, stream=None):
+    """perm [B, H, N] int32 of the reblocked layout (see bsa_reblock)."""
+    B, H, N, D = Q.shape
+    p = params(B, H, N, 1, prefix, D=D)
+    perm = torch.empty(B, H, N, dtype=torch.int32, device=Q.device)
+    ws = torch.empty(max(256, bsa_reblock_workspace_bytes(p)), dtype=torch.uint8, device=Q.device)
+    bsa_reblock(p, Q, K, perm, ws, stream)
+    return perm
+
+
+def forward_reblock(Q, K, V, top_k, prefix=0, variant="anchor", return_lse=False, ws=None,
+                    stream=None):
+    """bsa_forward_reblock: block-sparse attention on the reblocked layout,
+    O (and lse) returned in the original token order."""
+    B, H, N, D = Q.shape
+    p = params(B, H, N, top_k, prefix, variant, D=D)
+    O = torch.empty_like(Q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=Q.device) if return_lse else None
+    if ws is None:
+        ws = torch.empty(bsa_forward_reblock_workspace_bytes(p), dtype=torch.uint8,
+                         device=Q.device)
+    bsa_forward_reblock(p, Q, K, V, O, lse, ws, stream)
+    return (O, lse) if return_lse else O
 
 
 def bsa_fp8_operands_bytes(p: bsa_params) -> int:

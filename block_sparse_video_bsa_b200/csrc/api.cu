@@ -228,6 +228,83 @@ int attend_impl(const Shape& s, const void* Q, const void* K, const void* V, con
   return cuda_status(bsa::launch_attend(s, maps, idx, cnt, bias, O, lse, st));
 }
 
+// Reblocking scratch carved from one buffer (each piece 256-byte aligned).
+size_t reblock_carve(const Shape& s, const bsa::ReblockPlan& plan, uint8_t* base,
+                     bsa::ReblockBuffers* w) {
+  const size_t bh = static_cast<size_t>(s.B) * s.H;
+  const size_t nv = plan.nv;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += round256(bytes);
+    return p;
+  };
+  uint8_t* perm_tmp = take(bh * s.N * 4);
+  uint8_t* part = take(bh * plan.max_partials * 128 * 128 * 4);
+  uint8_t* psum = take(bh * plan.max_partials * 128 * 4);
+  uint8_t* vdir = take(bh * (static_cast<size_t>(1) << plan.levels) * 128 * 4);
+  uint8_t* r_hi = take(bh * 128 * 128 * 2);
+  uint8_t* r_lo = take(bh * 128 * 128 * 2);
+  uint8_t* u = take(bh * nv * 128 * 2);
+  uint8_t* keys = take(bh * nv * 4);
+  if (w) {
+    w->perm_tmp = reinterpret_cast<int32_t*>(perm_tmp);
+    w->part = reinterpret_cast<float*>(part);
+    w->psum = reinterpret_cast<float*>(psum);
+    w->vdir = reinterpret_cast<float*>(vdir);
+    w->r_hi = reinterpret_cast<__nv_bfloat16*>(r_hi);
+    w->r_lo = reinterpret_cast<__nv_bfloat16*>(r_lo);
+    w->u = reinterpret_cast<__nv_bfloat16*>(u);
+    w->keys = reinterpret_cast<uint32_t*>(keys);
+  }
+  return off;
+}
+
+int reblock_impl(const Shape& s, const void* Q, const void* K, int32_t* perm, uint8_t* ws,
+                 cudaStream_t st) {
+  const bsa::ReblockPlan plan = bsa::reblock_plan(s);
+  bsa::ReblockBuffers w;
+  reblock_carve(s, plan, ws, &w);
+  bsa::ReblockMaps maps;
+  const uint64_t bh = static_cast<uint64_t>(s.B) * s.H;
+  if (!make_map(&maps.q, Q, s.N, bh) || !make_map(&maps.r_hi, w.r_hi, 128, bh) ||
+      !make_map(&maps.r_lo, w.r_lo, 128, bh))
+    return BSA_ERR_UNSUPPORTED;
+  return cuda_status(bsa::launch_reblock(s, plan, Q, K, maps, w, perm, st));
+}
+
+// Workspace of bsa_forward_reblock: perm, the permuted Q/K/V/O and lse, the
+// reblocking scratch and the forward's own workspace.
+struct ReblockForwardWs {
+  int32_t* perm;
+  void *Qp, *Kp, *Vp, *Op;
+  float* lsep;
+  uint8_t* rb;
+  uint8_t* fw;
+};
+
+size_t reblock_forward_carve(const Shape& s, uint8_t* base, ReblockForwardWs* w) {
+  const size_t bh = static_cast<size_t>(s.B) * s.H;
+  const size_t rows = bh * s.N;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += round256(bytes);
+    return p;
+  };
+  uint8_t* perm = take(rows * 4);
+  uint8_t* qp = take(rows * 256);
+  uint8_t* kp = take(rows * 256);
+  uint8_t* vp = take(rows * 256);
+  uint8_t* op = take(rows * 256);
+  uint8_t* lsep = take(rows * 4);
+  uint8_t* rb = take(reblock_carve(s, bsa::reblock_plan(s), nullptr, nullptr));
+  uint8_t* fw = take(carve(s, nullptr, nullptr));
+  if (w) *w = ReblockForwardWs{reinterpret_cast<int32_t*>(perm), qp, kp, vp, op,
+                               reinterpret_cast<float*>(lsep), rb, fw};
+  return off;
+}
+
 int quantize_fp8_impl(const Shape& s, const void* Q, const void* K, const void* V,
                       const void* ksum, const void* vsum, const bsa::Fp8Operands& f,
                       cudaStream_t st) {
@@ -250,6 +327,92 @@ int attend_fp8_impl(const Shape& s, const bsa::Fp8Operands& f, const int32_t* id
 }  // namespace
 
 extern "C" {
+
+size_t bsa_reblock_workspace_bytes(const bsa_params* p) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK) return 0;
+  return reblock_carve(s, bsa::reblock_plan(s), nullptr, nullptr);
+}
+
+int bsa_reblock(const bsa_params* p, const void* Q, const void* K, int32_t* perm,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !K || !perm || !workspace) return BSA_ERR_INVALID;
+  if (workspace_bytes < reblock_carve(s, bsa::reblock_plan(s), nullptr, nullptr))
+    return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(perm, 4) || !aligned(workspace, 256))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return reblock_impl(s, Q, K, perm, static_cast<uint8_t*>(workspace),
+                      static_cast<cudaStream_t>(stream));
+}
+
+int bsa_permute(const bsa_params* p, const void* Q, const void* K, const void* V,
+                const int32_t* perm, void* Qp, void* Kp, void* Vp, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !K || !V || !perm || !Qp || !Kp || !Vp) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(Qp, 16) ||
+      !aligned(Kp, 16) || !aligned(Vp, 16) || !aligned(perm, 4))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return cuda_status(bsa::launch_permute_rows(s, Q, K, V, perm, Qp, Kp, Vp,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_unpermute(const bsa_params* p, const void* Op, const float* lsep, const int32_t* perm,
+                  void* O, float* lse, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Op || !perm || !O || (lse && !lsep)) return BSA_ERR_INVALID;
+  if (!aligned(Op, 16) || !aligned(O, 16) || !aligned(perm, 4) || (lse && !aligned(lse, 4)) ||
+      (lsep && !aligned(lsep, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return cuda_status(bsa::launch_unpermute_rows(s, Op, lse ? lsep : nullptr, perm, O, lse,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+size_t bsa_forward_reblock_workspace_bytes(const bsa_params* p) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK) return 0;
+  return reblock_forward_carve(s, nullptr, nullptr);
+}
+
+int bsa_forward_reblock(const bsa_params* p, const void* Q, const void* K, const void* V,
+                        void* O, float* lse, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !workspace) return BSA_ERR_INVALID;
+  if (workspace_bytes < reblock_forward_carve(s, nullptr, nullptr)) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
+      !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  ReblockForwardWs w;
+  reblock_forward_carve(s, static_cast<uint8_t*>(workspace), &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = reblock_impl(s, Q, K, w.perm, w.rb, st))) return rc;
+  if ((rc = cuda_status(bsa::launch_permute_rows(s, Q, K, V, w.perm, w.Qp, w.Kp, w.Vp, st))))
+    return rc;
+  Workspace fw;
+  carve(s, w.fw, &fw);
+  if ((rc = pool_impl(s, w.Qp, fw.qpool, fw.anchor, st))) return rc;
+  if ((rc = summarize_impl(s, w.Kp, w.Vp, fw.anchor, fw.kpool, fw.ksum, fw.vsum, fw.bias, st)))
+    return rc;
+  if ((rc = select_impl(s, fw.qpool, fw.kpool, fw.idx, fw.cnt, st))) return rc;
+  if ((rc = attend_impl(s, w.Qp, w.Kp, w.Vp, fw.idx, fw.cnt, fw.ksum, fw.vsum, fw.bias, w.Op,
+                        lse ? w.lsep : nullptr, st)))
+    return rc;
+  return cuda_status(
+      bsa::launch_unpermute_rows(s, w.Op, lse ? w.lsep : nullptr, w.perm, O, lse, st));
+}
 
 size_t bsa_fp8_operands_bytes(const bsa_params* p) {
   Shape s;

@@ -278,6 +278,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, ui
          | ((M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor, kind::f16: D fp32, A/B bf16, both MN-major (the
+// Gram of a tile of rows with itself: A = B = rows^T).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(uint32_t M, uint32_t N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) | ((N >> 3) << 17) |
+         ((M >> 4) << 24);
+}
+
 // Instruction descriptor, kind::f8f6f4: D fp32, A/B e4m3 (format code 0),
 // both K-major, M=128, N given.  K is 32 per instruction.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N) {

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace bsa {
@@ -58,6 +59,39 @@ struct AttendMapsFp8 {
 cudaError_t launch_attend_fp8(const Shape& s, const AttendMapsFp8& maps, const Fp8Operands& f,
                               const int32_t* idx, const float* bias, void* O, float* lse,
                               cudaStream_t st);
+
+// Adaptive reblocking (reblock.cu).  Tree shape of one call (depends on
+// N - prefix only): levels, chunk counts per level, partial-buffer slots.
+struct ReblockPlan {
+  int nv;                 // video tokens N - prefix
+  int levels;             // ceil(log2(ceil(nv / 128)))
+  int moment_chunks;      // 2048-row chunks of the key second moment
+  int max_partials;       // chunk partials per head (largest level)
+  int max_chunks[16];     // 2048-row chunks of the largest group, per level
+  int max_pchunks[16];    // 512-position projection chunks of the largest group
+};
+ReblockPlan reblock_plan(const Shape& s);
+struct ReblockBuffers {
+  int32_t* perm_tmp;      // [BH, N]
+  float* part;            // [BH, max_partials, 128, 128]
+  float* psum;            // [BH, max_partials, 128]
+  float* vdir;            // [BH, 2^levels, 128]
+  __nv_bfloat16* r_hi;    // [BH, 128, 128]
+  __nv_bfloat16* r_lo;    // [BH, 128, 128]
+  __nv_bfloat16* u;       // [BH, nv, 128]
+  uint32_t* keys;         // [BH, nv]
+};
+struct ReblockMaps {
+  CUtensorMap q, r_hi, r_lo;   // bf16, box {64, 128, 1}, 128B swizzle
+};
+cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* Q, const void* K,
+                           const ReblockMaps& maps, const ReblockBuffers& w, int32_t* perm_out,
+                           cudaStream_t st);
+cudaError_t launch_permute_rows(const Shape& s, const void* Q, const void* K, const void* V,
+                                const int32_t* perm, void* Qp, void* Kp, void* Vp,
+                                cudaStream_t st);
+cudaError_t launch_unpermute_rows(const Shape& s, const void* Op, const float* lsep,
+                                  const int32_t* perm, void* O, float* lse, cudaStream_t st);
 
 cudaError_t launch_expired_wait(int32_t* dev_status, uint64_t timeout_ns, cudaStream_t st);
 

@@ -1,0 +1,738 @@
+// Adaptive reblocking of the query/key layout (Spark-Reblock).
+//
+// Spark-H3 page, section "What Spark-Attn changes", Spark-Reblock bullet: two
+// queries are similar when their attention-score patterns over the keys are
+// similar (a Mahalanobis cosine induced by the keys' second moment), and a
+// hierarchical partitioner splits groups until every leaf holds one block, in
+// O(N log N); section "Workflows": keys reuse the query layout (q_reuse_k).
+// This library's reading (the pages give no formulas):
+//   M = sum_{t >= P} k_t k_t^T;  L L^T = M + 1e-6 * trace(M) / 128 * I;
+//   u_t = L^T q_t / |L^T q_t|  (so u . u' is the cosine of the score vectors);
+//   a group of n tokens (b = ceil(n/128) >= 2 blocks) is bisected along its
+//   principal axis: c = mean u, v = 8 power iterations of the centred scatter
+//   sum (u - c)(u - c)^T from (1, ..., 1)/sqrt(128), p = u . v; the
+//   floor(b/2)*128 tokens of smallest p (ties to the lower original index) go
+//   left.  Leaves are laid out left to right, ascending inside a leaf; the
+//   dense prefix rows [0, P) stay in place.
+//
+// Kernels (all heads of a call at once):
+//   gram_kernel<moment>   sum x x^T over the video keys, chunks of 2048 rows:
+//                         rows staged through shared memory in the 128-byte
+//                         swizzled layout, tcgen05.mma with A = B = rows^T
+//                         (MN-major), fp32 accumulator in TMEM; partials per
+//                         chunk, reduced in a fixed order by factor_kernel.
+//   factor_kernel         Cholesky of M (fp64, one CTA per head); writes
+//                         R = L^T as bf16 hi + lo (R ~= hi + lo to ~16 bits).
+//   whiten_kernel         Y = Q R^T on tcgen05 (two MMAs per K step: hi, lo),
+//                         u = Y / |Y| stored bf16, one CTA per 128 tokens.
+//   per level (group j of level l found by descending the tree; the groups
+//   of a level are ranges of the working order `perm`):
+//   gram_kernel<group>    sum u u^T and sum u over a chunk of a group's
+//                         rows (gathered through perm); a group that fits in
+//                         one chunk finishes its power iteration in the same
+//                         CTA, larger groups leave partials for group_kernel.
+//   group_kernel          fixed-order sum of a large group's partials, power
+//                         iteration.
+//   project_kernel        p = u . v per position -> order-preserving key.
+//   split_kernel          radix select of the floor(b/2)*128-th key (four
+//                         8-bit passes over the group's keys, ties broken by
+//                         position), then a stable partition of perm.
+//   permute / unpermute   row gathers of Q, K, V into the new layout and the
+//                         scatter of O and lse back.
+// Every wait is bounded (globaltimer); on expiry the CTA records
+// BSA_ERR_TIMEOUT, drains its MMAs, frees TMEM and returns.
+#include "bsa_device.cuh"
+#include "bsa_kernels.h"
+
+namespace bsa {
+
+namespace {
+
+constexpr int kChunkTok = 2048;   // rows per Gram chunk (16 tiles)
+constexpr int kProjTok = 512;     // positions per projection CTA
+constexpr int kPowerIters = 8;
+constexpr uint32_t kTile = 32768;          // 128 rows x 128 bf16
+constexpr uint32_t kHalf = 16384;          // one 64-column swizzle-atom-wide box
+
+struct Range {
+  int start, count;
+};
+
+// Group j of level `level`: descend from the root (count <= 128 is a leaf,
+// so its descendants do not exist: count 0).
+__device__ __forceinline__ Range group_of(int nv, int level, int j) {
+  int start = 0, count = nv;
+  for (int k = 0; k < level; ++k) {
+    if (count <= kBlock) return {0, 0};
+    const int m = ((count + kBlock - 1) / kBlock / 2) * kBlock;
+    if ((j >> (level - 1 - k)) & 1) {
+      start += m;
+      count -= m;
+    } else {
+      count = m;
+    }
+  }
+  return {start, count};
+}
+
+// 16-byte chunk c16 (0..15) of row r of a 128 x 128 bf16 tile in the 128-byte
+// swizzled layout (two 64-column boxes, rows of 128 bytes, chunk index XOR
+// row % 8): the layout the MN-major shared-memory descriptors below expect.
+__device__ __forceinline__ uint32_t swz(int r, int c16) {
+  return static_cast<uint32_t>((c16 >> 3) * kHalf + r * 128 + ((((c16 & 7) ^ (r & 7))) << 4));
+}
+
+// 128 threads, thread i owns row i of G (in g[]); smem v[128], c[128] (mean),
+// red[4].  Writes the unit direction of kPowerIters iterations of
+// C = G - n c c^T from (1, ..., 1)/sqrt(128) to out[i].  A zero step keeps v.
+__device__ __forceinline__ void power_iterate(const float (&g)[128], float n, float* c, float* v,
+                                              float* red, float* out) {
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  v[i] = 0.08838834764831845f;   // 1 / sqrt(128)
+  __syncthreads();
+  for (int it = 0; it < kPowerIters; ++it) {
+    float cv = 0.f, w = 0.f;
+#pragma unroll   // fully: g[] stays in registers
+    for (int j = 0; j < 128; ++j) {
+      cv = fmaf(c[j], v[j], cv);
+      w = fmaf(g[j], v[j], w);
+    }
+    w = fmaf(-n * c[i], cv, w);
+    float s = w * w;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) red[warp] = s;
+    __syncthreads();
+    const float tot = (red[0] + red[1]) + (red[2] + red[3]);
+    if (tot > 0.f) v[i] = w / sqrtf(tot);
+    __syncthreads();
+    if (!(tot > 0.f)) break;
+  }
+  out[i] = v[i];
+}
+
+struct GramArgs {
+  const __nv_bfloat16* X;   // moment: K [BH, N, 128]; group: u [BH, nv, 128]
+  const int32_t* perm;      // group mode: [BH, N] working order (original indices)
+  int N, prefix, nv;
+  int level, slots, max_chunks;
+  float* part;              // [BH, slots * max_chunks, 128, 128]
+  float* psum;              // [BH, slots * max_chunks, 128]  (group mode)
+  float* vdir;              // [BH, slots, 128]                (group mode)
+  int* dev_status;
+};
+
+struct GramSmem {
+  uint64_t done[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  float c[128], v[128], red[4];
+};
+
+template <bool kGroup>
+__global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  GramSmem* ctl = reinterpret_cast<GramSmem*>(sm + 2 * kTile);
+  const int tid = threadIdx.x;
+  const size_t bh = blockIdx.y;
+  int slot = 0, chunk = blockIdx.x, p0, p1;
+  Range g{0, a.nv};
+  if constexpr (kGroup) {
+    slot = blockIdx.x / a.max_chunks;
+    chunk = blockIdx.x - slot * a.max_chunks;
+    g = group_of(a.nv, a.level, slot);
+    if (g.count <= kBlock) return;
+  }
+  p0 = g.start + chunk * kChunkTok;
+  p1 = min(p0 + kChunkTok, g.start + g.count);
+  if (p0 >= p1) return;
+  const bool single = kGroup && g.count <= kChunkTok;
+  if ((smem_u32(sm) & 1023u) != 0) {   // the swizzled layout needs 1024-byte alignment
+    if (tid == 0 && a.dev_status) atomicExch(a.dev_status, kErrTimeout);
+    return;
+  }
+
+  if (tid == 0) {
+    mbar_init(&ctl->done[0], 1);
+    mbar_init(&ctl->done[1], 1);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (tid < 32) {
+    tmem_alloc(&ctl->tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const WaitCtx wc{&ctl->abort_flag, a.dev_status};
+  const uint32_t idesc = idesc_bf16_f32_mn(128, 128);
+
+  auto row_ptr = [&](int pos) -> const __nv_bfloat16* {
+    if constexpr (kGroup) {
+      const int orig = __ldg(a.perm + bh * a.N + a.prefix + pos);
+      return a.X + (bh * a.nv + (orig - a.prefix)) * kDim;
+    } else {
+      return a.X + (bh * a.N + a.prefix + pos) * kDim;
+    }
+  };
+
+  const int ntile = (p1 - p0 + kBlock - 1) / kBlock;
+  float colsum = 0.f;
+  bool ok = true;
+  for (int it = 0; it < ntile && ok; ++it) {
+    const int b = it & 1;
+    if (it >= 2 && !mbar_wait(&ctl->done[b], ((it - 2) >> 1) & 1, wc)) { ok = false; break; }
+    uint8_t* buf = sm + b * kTile;
+    const int base = p0 + it * kBlock;
+    const int nrow = min(kBlock, p1 - base);
+#pragma unroll 4
+    for (int ps = 0; ps < 16; ++ps) {
+      const int r = ps * 8 + (tid >> 4), c16 = tid & 15;
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (r < nrow) w = ld_stream_v4(reinterpret_cast<const uint4*>(row_ptr(base + r)) + c16);
+      *reinterpret_cast<uint4*>(buf + swz(r, c16)) = w;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if constexpr (kGroup) {   // column tid of the tile's rows
+      const int c16 = tid >> 3, e = tid & 7;
+      for (int r = 0; r < nrow; ++r)
+        colsum += __bfloat162float(
+            *reinterpret_cast<const __nv_bfloat16*>(buf + swz(r, c16) + 2 * e));
+    }
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t addr = smem_u32(buf);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {   // 16 rows per MMA
+        const uint64_t d = smem_desc_sw128(addr + kk * 2048, kHalf, 1024);
+        mma_bf16_ss(tmem, d, d, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(&ctl->done[b]);
+    }
+  }
+  // the last tile's MMAs (all earlier ones complete in order before it)
+  const int last = ntile - 1;
+  if (ok && !mbar_wait(&ctl->done[last & 1], (last >> 1) & 1, wc)) ok = false;
+  ok = __syncthreads_and(ok);
+  tc_fence_after();
+
+  if (ok) {
+    const uint32_t lane_base = static_cast<uint32_t>((tid >> 5) * 32) << 16;
+    float gr[128];
+    BSA_TMEM_LD_32F(tmem + lane_base, gr);
+    BSA_TMEM_LD_32F(tmem + lane_base + 32, gr + 32);
+    BSA_TMEM_LD_32F(tmem + lane_base + 64, gr + 64);
+    BSA_TMEM_LD_32F(tmem + lane_base + 96, gr + 96);
+    tmem_wait_ld();
+    const size_t pidx = static_cast<size_t>(bh) * a.slots * a.max_chunks +
+                        static_cast<size_t>(slot) * a.max_chunks + chunk;
+    if (single) {
+      const float n = static_cast<float>(g.count);
+      ctl->c[tid] = colsum / n;
+      __syncthreads();
+      power_iterate(gr, n, ctl->c, ctl->v, ctl->red,
+                    a.vdir + (bh * a.slots + slot) * kDim);
+    } else {
+      float4* dst = reinterpret_cast<float4*>(a.part + (pidx * 128 + tid) * 128);
+#pragma unroll
+      for (int q = 0; q < 32; ++q)
+        dst[q] = make_float4(gr[4 * q], gr[4 * q + 1], gr[4 * q + 2], gr[4 * q + 3]);
+      if constexpr (kGroup) a.psum[pidx * 128 + tid] = colsum;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid < 32) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// Power iteration of a group larger than one chunk: fixed-order sum of its
+// chunk partials.
+__global__ void __launch_bounds__(128) group_kernel(const GramArgs a) {
+  __shared__ float c[128], v[128], red[4];
+  const int tid = threadIdx.x, slot = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  const Range g = group_of(a.nv, a.level, slot);
+  if (g.count <= kChunkTok) return;   // leaves and single-chunk groups are done
+  const int nch = (g.count + kChunkTok - 1) / kChunkTok;
+  float gr[128];
+#pragma unroll
+  for (int j = 0; j < 128; ++j) gr[j] = 0.f;
+  float s = 0.f;
+  const size_t p0 = static_cast<size_t>(bh) * a.slots * a.max_chunks +
+                    static_cast<size_t>(slot) * a.max_chunks;
+  for (int ch = 0; ch < nch; ++ch) {
+    const float4* src = reinterpret_cast<const float4*>(a.part + ((p0 + ch) * 128 + tid) * 128);
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const float4 x = src[q];
+      gr[4 * q] += x.x;
+      gr[4 * q + 1] += x.y;
+      gr[4 * q + 2] += x.z;
+      gr[4 * q + 3] += x.w;
+    }
+    s += a.psum[(p0 + ch) * 128 + tid];
+  }
+  const float n = static_cast<float>(g.count);
+  c[tid] = s / n;
+  __syncthreads();
+  power_iterate(gr, n, c, v, red, a.vdir + (bh * a.slots + slot) * kDim);
+}
+
+// Cholesky of the key second moment (fp64, in shared memory, lower triangle
+// in place) and R = L^T split into bf16 hi + lo.
+__global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ part, int nchunk,
+                                                     __nv_bfloat16* __restrict__ r_hi,
+                                                     __nv_bfloat16* __restrict__ r_lo) {
+  extern __shared__ double M[];   // [128][129]
+  __shared__ double red[128];
+  const int tid = threadIdx.x;
+  const size_t bh = blockIdx.x;
+  constexpr int ld = 129;
+  for (int i = 0; i < 128; ++i) {   // column tid of row i (coalesced)
+    double s = 0.0;
+    for (int ch = 0; ch < nchunk; ++ch)
+      s += part[((bh * nchunk + ch) * 128 + i) * 128 + tid];
+    M[i * ld + tid] = s;
+  }
+  __syncthreads();
+  red[tid] = M[tid * ld + tid];
+  __syncthreads();
+  if (tid == 0) {
+    double tr = 0.0;
+    for (int i = 0; i < 128; ++i) tr += red[i];
+    red[0] = 1e-6 * tr / 128.0;
+  }
+  __syncthreads();
+  const double ridge = red[0];
+  M[tid * ld + tid] += ridge;
+  __syncthreads();
+  for (int j = 0; j < 128; ++j) {
+    if (tid == 0) {
+      double s = M[j * ld + j];
+      for (int k = 0; k < j; ++k) s -= M[j * ld + k] * M[j * ld + k];
+      M[j * ld + j] = sqrt(s > 0.0 ? s : 1e-300);
+    }
+    __syncthreads();
+    if (tid > j) {
+      double s = M[tid * ld + j];
+      for (int k = 0; k < j; ++k) s -= M[tid * ld + k] * M[j * ld + k];
+      M[tid * ld + j] = s / M[j * ld + j];
+    }
+    __syncthreads();
+  }
+  // R = L^T: R[i][j] = L[j][i] for j >= i; thread tid writes column j = tid
+  for (int i = 0; i < 128; ++i) {
+    const float r = tid >= i ? static_cast<float>(M[tid * ld + i]) : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(r);
+    r_hi[(bh * 128 + i) * 128 + tid] = hi;
+    r_lo[(bh * 128 + i) * 128 + tid] = __float2bfloat16_rn(r - __bfloat162float(hi));
+  }
+}
+
+struct WhitenSmem {
+  uint64_t full, done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// u = Y / |Y|, Y = Q R^T (R ~= hi + lo), one CTA per 128 video tokens.
+__global__ void __launch_bounds__(128) whiten_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                     const __grid_constant__ CUtensorMap tm_hi,
+                                                     const __grid_constant__ CUtensorMap tm_lo,
+                                                     int prefix, int nv,
+                                                     __nv_bfloat16* __restrict__ u,
+                                                     int* dev_status) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  WhitenSmem* ctl = reinterpret_cast<WhitenSmem*>(sm + 3 * kTile);
+  const int tid = threadIdx.x;
+  const int tile = blockIdx.x;
+  const int bh = blockIdx.y;
+  if ((smem_u32(sm) & 1023u) != 0) {
+    if (tid == 0 && dev_status) atomicExch(dev_status, kErrTimeout);
+    return;
+  }
+  if (tid == 0) {
+    mbar_init(&ctl->full, 1);
+    mbar_init(&ctl->done, 1);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (tid < 32) {
+    tmem_alloc(&ctl->tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const WaitCtx wc{&ctl->abort_flag, dev_status};
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&ctl->full, 3 * kTile);
+    const int row = prefix + tile * kBlock;
+    tma_load_3d(sm, &tm_q, &ctl->full, 0, row, bh);
+    tma_load_3d(sm + kHalf, &tm_q, &ctl->full, 64, row, bh);
+    tma_load_3d(sm + kTile, &tm_hi, &ctl->full, 0, 0, bh);
+    tma_load_3d(sm + kTile + kHalf, &tm_hi, &ctl->full, 64, 0, bh);
+    tma_load_3d(sm + 2 * kTile, &tm_lo, &ctl->full, 0, 0, bh);
+    tma_load_3d(sm + 2 * kTile + kHalf, &tm_lo, &ctl->full, 64, 0, bh);
+  }
+  bool ok = mbar_wait(&ctl->full, 0, wc);
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    const uint32_t id = idesc_bf16_f32(128, 128, 0);
+    const uint32_t q = smem_u32(sm);
+    for (int part = 0; part < 2; ++part) {
+      const uint32_t rr = smem_u32(sm + (1 + part) * kTile);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+        mma_bf16_ss(tmem, smem_desc_sw128(q + off, 16, 1024), smem_desc_sw128(rr + off, 16, 1024),
+                    id, (part > 0 || kk > 0) ? 1u : 0u);
+      }
+    }
+    mma_commit(&ctl->done);
+  }
+  ok = __syncthreads_and(ok);
+  if (ok) ok = mbar_wait(&ctl->done, 0, wc);
+  ok = __syncthreads_and(ok);
+  tc_fence_after();
+  if (ok) {
+    const uint32_t lane_base = static_cast<uint32_t>((tid >> 5) * 32) << 16;
+    float y[128];
+    BSA_TMEM_LD_32F(tmem + lane_base, y);
+    BSA_TMEM_LD_32F(tmem + lane_base + 32, y + 32);
+    BSA_TMEM_LD_32F(tmem + lane_base + 64, y + 64);
+    BSA_TMEM_LD_32F(tmem + lane_base + 96, y + 96);
+    tmem_wait_ld();
+    const int t = tile * kBlock + tid;
+    if (t < nv) {
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < 128; ++j) ss = fmaf(y[j], y[j], ss);
+      const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(u + (static_cast<size_t>(bh) * nv + t) * kDim);
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        dst[q] = make_uint4(pack_bf16x2(y[8 * q] * inv, y[8 * q + 1] * inv),
+                            pack_bf16x2(y[8 * q + 2] * inv, y[8 * q + 3] * inv),
+                            pack_bf16x2(y[8 * q + 4] * inv, y[8 * q + 5] * inv),
+                            pack_bf16x2(y[8 * q + 6] * inv, y[8 * q + 7] * inv));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid < 32) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// p = u . v (16 lanes per row, fixed order), stored as an order-preserving key.
+__global__ void __launch_bounds__(256) project_kernel(const __nv_bfloat16* __restrict__ u,
+                                                      const int32_t* __restrict__ perm,
+                                                      const float* __restrict__ vdir, int N,
+                                                      int prefix, int nv, int level, int slots,
+                                                      int max_pchunks,
+                                                      uint32_t* __restrict__ keys) {
+  __shared__ float v[128];
+  const int tid = threadIdx.x;
+  const int slot = blockIdx.x / max_pchunks, chunk = blockIdx.x - slot * max_pchunks;
+  const size_t bh = blockIdx.y;
+  const Range g = group_of(nv, level, slot);
+  if (g.count <= kBlock) return;
+  const int p0 = g.start + chunk * kProjTok, p1 = min(p0 + kProjTok, g.start + g.count);
+  if (p0 >= p1) return;
+  if (tid < 128) v[tid] = vdir[(bh * slots + slot) * kDim + tid];
+  __syncthreads();
+  const int c16 = tid & 15;
+  float vv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) vv[e] = v[8 * c16 + e];
+  // every half-warp runs the same number of iterations (the shuffles below
+  // span the whole warp); the tail masks the load instead
+  for (int base = p0; base < p1; base += 16) {
+    const int pos = base + (tid >> 4);
+    const bool valid = pos < p1;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (valid) {
+      const int orig = __ldg(perm + bh * N + prefix + pos);
+      w = ld_stream_v4(reinterpret_cast<const uint4*>(u + (bh * nv + (orig - prefix)) * kDim) +
+                       c16);
+    }
+    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&w);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s = fmaf(__bfloat162float(h[e]), vv[e], s);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (valid && c16 == 0) keys[bh * nv + pos] = orderable_key(s);
+  }
+}
+
+// Exclusive block-wide scan of one int per thread (512 threads); returns the
+// thread's prefix and writes the block total to *total.
+__device__ __forceinline__ int block_scan(int x, int* wsum, int* total) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int w = 0; w < 16; ++w) {
+      const int t = wsum[w];
+      wsum[w] = run;
+      run += t;
+    }
+    *total = run;
+  }
+  __syncthreads();
+  const int res = wsum[warp] + incl - x;
+  __syncthreads();
+  return res;
+}
+
+// Radix select of the m-th smallest key of a group (m = floor(b/2) * 128;
+// equal keys count in position order), then the stable partition of perm.
+__global__ void __launch_bounds__(512) split_kernel(const uint32_t* __restrict__ keys,
+                                                    const int32_t* __restrict__ perm_in,
+                                                    int32_t* __restrict__ perm_out, int N,
+                                                    int prefix, int nv, int level) {
+  __shared__ int hist[256];
+  __shared__ int wsum[16];
+  __shared__ int sh[4];
+  const int tid = threadIdx.x;
+  const size_t bh = blockIdx.y;
+  const Range g = group_of(nv, level, blockIdx.x);
+  if (g.count <= kBlock) return;
+  const int m = ((g.count + kBlock - 1) / kBlock / 2) * kBlock;
+  const uint32_t* k = keys + bh * nv + g.start;
+  uint32_t prefix_bits = 0, mask = 0;
+  int want = m;   // rank (1-based) of the wanted key among those matching the prefix
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += 512) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < g.count; i += 512) {
+      const uint32_t x = __ldg(k + i);
+      if ((x & mask) == prefix_bits) atomicAdd(&hist[(x >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0, d = 0;
+      for (d = 0; d < 255; ++d) {
+        if (run + hist[d] >= want) break;
+        run += hist[d];
+      }
+      sh[0] = d;
+      sh[1] = want - run;
+    }
+    __syncthreads();
+    prefix_bits |= static_cast<uint32_t>(sh[0]) << shift;
+    mask |= 255u << shift;
+    want = sh[1];
+    __syncthreads();
+  }
+  const uint32_t T = prefix_bits;   // the m-th smallest key
+  const int need_eq = want;         // equal keys (in position order) that go left
+  int left_run = 0, eq_run = 0;
+  const int32_t* pin = perm_in + bh * N + prefix + g.start;
+  int32_t* pout = perm_out + bh * N + prefix + g.start;
+  for (int base = 0; base < g.count; base += 512) {
+    const int i = base + tid;
+    const bool valid = i < g.count;
+    const uint32_t x = valid ? __ldg(k + i) : 0xffffffffu;
+    const int eq = (valid && x == T) ? 1 : 0;
+    int eq_tot;
+    const int eq_before = eq_run + block_scan(eq, wsum, &sh[2]);
+    eq_tot = sh[2];
+    const int left = (valid && (x < T || (eq && eq_before < need_eq))) ? 1 : 0;
+    const int l_before = left_run + block_scan(left, wsum, &sh[3]);
+    const int l_tot = sh[3];
+    if (valid) {
+      const int dst = left ? l_before : m + (i - l_before);
+      pout[dst] = pin[i];
+    }
+    left_run += l_tot;
+    eq_run += eq_tot;
+    __syncthreads();
+  }
+}
+
+__global__ void init_perm_kernel(int32_t* __restrict__ perm, int N) {
+  const size_t bh = blockIdx.y;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < N; t += gridDim.x * blockDim.x)
+    perm[bh * N + t] = t;
+}
+
+// Xp[bh][i] = X[bh][perm[bh][i]] for Q, K, V (16 lanes per 256-byte row).
+__global__ void __launch_bounds__(256) permute_rows_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                           const __nv_bfloat16* __restrict__ K,
+                                                           const __nv_bfloat16* __restrict__ V,
+                                                           const int32_t* __restrict__ perm,
+                                                           int N, __nv_bfloat16* __restrict__ Qp,
+                                                           __nv_bfloat16* __restrict__ Kp,
+                                                           __nv_bfloat16* __restrict__ Vp) {
+  const size_t bh = blockIdx.y;
+  const int c16 = threadIdx.x & 15;
+  for (int i = blockIdx.x * 16 + (threadIdx.x >> 4); i < N; i += gridDim.x * 16) {
+    const size_t src = (bh * N + __ldg(perm + bh * N + i)) * kDim;
+    const size_t dst = (bh * N + i) * kDim;
+    reinterpret_cast<uint4*>(Qp + dst)[c16] = ld_stream_v4(reinterpret_cast<const uint4*>(Q + src) + c16);
+    reinterpret_cast<uint4*>(Kp + dst)[c16] = ld_stream_v4(reinterpret_cast<const uint4*>(K + src) + c16);
+    reinterpret_cast<uint4*>(Vp + dst)[c16] = ld_stream_v4(reinterpret_cast<const uint4*>(V + src) + c16);
+  }
+}
+
+// O[bh][perm[bh][i]] = Op[bh][i] (and lse).
+__global__ void __launch_bounds__(256) unpermute_rows_kernel(const __nv_bfloat16* __restrict__ Op,
+                                                             const float* __restrict__ lsep,
+                                                             const int32_t* __restrict__ perm,
+                                                             int N, __nv_bfloat16* __restrict__ O,
+                                                             float* __restrict__ lse) {
+  const size_t bh = blockIdx.y;
+  const int c16 = threadIdx.x & 15;
+  for (int i = blockIdx.x * 16 + (threadIdx.x >> 4); i < N; i += gridDim.x * 16) {
+    const int t = __ldg(perm + bh * N + i);
+    reinterpret_cast<uint4*>(O + (bh * N + t) * kDim)[c16] =
+        ld_stream_v4(reinterpret_cast<const uint4*>(Op + (bh * N + i) * kDim) + c16);
+    if (lse && c16 == 0) lse[bh * N + t] = lsep[bh * N + i];
+  }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host side
+
+ReblockPlan reblock_plan(const Shape& s) {
+  ReblockPlan p;
+  p.nv = s.N - s.prefix;
+  p.levels = 0;
+  while ((kBlock << p.levels) < p.nv) ++p.levels;   // ceil(log2(ceil(nv / 128)))
+  p.moment_chunks = (p.nv + kChunkTok - 1) / kChunkTok;
+  p.max_partials = 1;
+  int largest = p.nv;   // the rightmost group is the largest of its level
+  for (int l = 0; l < p.levels; ++l) {
+    const int chunks = (largest + kChunkTok - 1) / kChunkTok;
+    p.max_chunks[l] = chunks;
+    p.max_pchunks[l] = (largest + kProjTok - 1) / kProjTok;
+    const long long parts = (chunks > 1) ? (static_cast<long long>(1) << l) * chunks : 1;
+    if (parts > p.max_partials) p.max_partials = static_cast<int>(parts);
+    const int m = ((largest + kBlock - 1) / kBlock / 2) * kBlock;
+    largest -= m;
+  }
+  if (p.moment_chunks > p.max_partials) p.max_partials = p.moment_chunks;
+  return p;
+}
+
+cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* Q, const void* K,
+                           const ReblockMaps& maps, const ReblockBuffers& w, int32_t* perm_out,
+                           cudaStream_t st) {
+  const int BH = s.B * s.H;
+  const int nv = plan.nv;
+  // Gram kernels: two 32 KB tiles + control; factor: 128 x 129 doubles.
+  const size_t gram_smem = 2 * kTile + sizeof(GramSmem) + 1024;
+  const size_t whiten_smem = 3 * kTile + sizeof(WhitenSmem) + 1024;
+  const size_t factor_smem = 128 * 129 * sizeof(double);
+  static bool attr[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr[dev]) {
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(gram_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  gram_smem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(gram_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  gram_smem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(whiten_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  whiten_smem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  factor_smem)) != cudaSuccess)
+      return e;
+    attr[dev] = true;
+  }
+  int32_t* pa = perm_out;
+  int32_t* pb = w.perm_tmp;
+  init_perm_kernel<<<dim3(64, BH), 256, 0, st>>>(pa, s.N);
+  if (plan.levels == 0) return cudaGetLastError();
+
+  GramArgs ga{};
+  ga.N = s.N;
+  ga.prefix = s.prefix;
+  ga.nv = nv;
+  ga.part = w.part;
+  ga.psum = w.psum;
+  ga.vdir = w.vdir;
+  ga.dev_status = s.dev_status;
+  // 1. key second moment (chunk partials), 2. factor, 3. whiten
+  ga.X = static_cast<const __nv_bfloat16*>(K);
+  ga.perm = nullptr;
+  ga.level = 0;
+  ga.slots = 1;
+  ga.max_chunks = plan.moment_chunks;
+  gram_kernel<false><<<dim3(plan.moment_chunks, BH), 128, gram_smem, st>>>(ga);
+  factor_kernel<<<BH, 128, factor_smem, st>>>(w.part, plan.moment_chunks, w.r_hi, w.r_lo);
+  whiten_kernel<<<dim3((nv + kBlock - 1) / kBlock, BH), 128, whiten_smem, st>>>(
+      maps.q, maps.r_hi, maps.r_lo, s.prefix, nv, w.u, s.dev_status);
+  (void)Q;
+  // 4. levels
+  ga.X = w.u;
+  for (int l = 0; l < plan.levels; ++l) {
+    const int slots = 1 << l;
+    cudaError_t e = cudaMemcpyAsync(pb, pa, static_cast<size_t>(BH) * s.N * sizeof(int32_t),
+                                    cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return e;
+    ga.perm = pa;
+    ga.level = l;
+    ga.slots = slots;
+    ga.max_chunks = plan.max_chunks[l];
+    gram_kernel<true><<<dim3(slots * plan.max_chunks[l], BH), 128, gram_smem, st>>>(ga);
+    if (plan.max_chunks[l] > 1) group_kernel<<<dim3(slots, BH), 128, 0, st>>>(ga);
+    project_kernel<<<dim3(slots * plan.max_pchunks[l], BH), 256, 0, st>>>(
+        w.u, pa, w.vdir, s.N, s.prefix, nv, l, slots, plan.max_pchunks[l], w.keys);
+    split_kernel<<<dim3(slots, BH), 512, 0, st>>>(w.keys, pa, pb, s.N, s.prefix, nv, l);
+    int32_t* t = pa;
+    pa = pb;
+    pb = t;
+  }
+  if (pa != perm_out) {
+    cudaError_t e = cudaMemcpyAsync(perm_out, pa, static_cast<size_t>(BH) * s.N * sizeof(int32_t),
+                                    cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_rows(const Shape& s, const void* Q, const void* K, const void* V,
+                                const int32_t* perm, void* Qp, void* Kp, void* Vp,
+                                cudaStream_t st) {
+  const int BH = s.B * s.H;
+  const int blocks = (s.N + 15) / 16 < 1024 ? (s.N + 15) / 16 : 1024;
+  permute_rows_kernel<<<dim3(blocks, BH), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
+      static_cast<const __nv_bfloat16*>(V), perm, s.N, static_cast<__nv_bfloat16*>(Qp),
+      static_cast<__nv_bfloat16*>(Kp), static_cast<__nv_bfloat16*>(Vp));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpermute_rows(const Shape& s, const void* Op, const float* lsep,
+                                  const int32_t* perm, void* O, float* lse, cudaStream_t st) {
+  const int BH = s.B * s.H;
+  const int blocks = (s.N + 15) / 16 < 1024 ? (s.N + 15) / 16 : 1024;
+  unpermute_rows_kernel<<<dim3(blocks, BH), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(Op), lsep, perm, s.N, static_cast<__nv_bfloat16*>(O),
+      lse);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

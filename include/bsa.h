@@ -190,6 +190,52 @@ int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK,
 int bsa_forward_noalloc(const bsa_params* p, const void* Q, const void* K, const void* V,
                         void* O, float* lse, void* stream);
 
+/* ---- adaptive reblocking (Spark-Reblock) ------------------------------ */
+
+/* Spark-H3 page, section "What Spark-Attn changes", Spark-Reblock bullet:
+ * the fixed token blocks are replaced by an adaptive partition in which two
+ * queries are similar when their score patterns over the keys are similar (a
+ * Mahalanobis cosine induced by the keys' second moment); a hierarchical
+ * partitioner splits groups down to one block, in O(N log N).  Section
+ * "Workflows": keys reuse the query layout (q_reuse_k).  This library's
+ * reading:
+ *   M = sum_{t >= prefix} k_t k_t^T, L L^T = M + 1e-6 * trace(M) / 128 * I,
+ *   u_t = L^T q_t / |L^T q_t| (u . u' = cosine of the two score vectors);
+ *   a group of n tokens with b = ceil(n/128) >= 2 blocks is bisected along
+ *   its principal axis (8 power iterations of the centred scatter of u from
+ *   the all-ones direction): the floor(b/2) * 128 tokens of smallest
+ *   projection go left (ties to the lower original index);
+ *   leaves left to right, ascending inside a leaf; prefix rows stay put.
+ * The GPU stores u in bf16, so tokens within ~2^-9 of a split's threshold may
+ * land on either side of it. */
+
+/* Scratch of bsa_reblock (device, caller-owned, 256-byte aligned). */
+size_t bsa_reblock_workspace_bytes(const bsa_params* p);
+
+/* perm (int32 [B,H,N], caller-owned): perm[b,h,i] = the original index of the
+ * token at position i of the reblocked layout. */
+int bsa_reblock(const bsa_params* p, const void* Q, const void* K, int32_t* perm,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Qp[b,h,i] = Q[b,h,perm[b,h,i]] (and K, V): the reblocked layout. */
+int bsa_permute(const bsa_params* p, const void* Q, const void* K, const void* V,
+                const int32_t* perm, void* Qp, void* Kp, void* Vp, void* stream);
+
+/* O[b,h,perm[b,h,i]] = Op[b,h,i] (and lse from lsep when lse is non-NULL):
+ * back to the original token order. */
+int bsa_unpermute(const bsa_params* p, const void* Op, const float* lsep, const int32_t* perm,
+                  void* O, float* lse, void* stream);
+
+/* Workspace of bsa_forward_reblock: perm, the reblocked Q/K/V/O and lse, the
+ * reblocking scratch and the forward's workspace. */
+size_t bsa_forward_reblock_workspace_bytes(const bsa_params* p);
+
+/* bsa_reblock, bsa_permute, bsa_forward (pool, summarize, select, attend) on
+ * the reblocked layout, bsa_unpermute: O (and lse) in the original order. */
+int bsa_forward_reblock(const bsa_params* p, const void* Q, const void* K, const void* V,
+                        void* O, float* lse, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
 /* ---- FP8 (e4m3) exact and compressed branch --------------------------- */
 
 /* The pages name a quantised sparse kernel ("H3 Sparse Attention", comfy.icu
