@@ -2,11 +2,14 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload h3_768p_5s] [--top-k K] [--no-cpu-baseline] [--no-e2e]
-                    [--precision bf16|fp8]
+                    [--precision bf16|fp8] [--reblock]
 
 One step = one whole attention call (pool -> summarize -> select -> attend,
 all through the C ABI) over one batch of synthetic bf16 input of the 768p-5s
 H3 shape (B=1, H=56, N=37,740, d=128, top_k=64, anchor-weighted summaries).
+``--reblock`` times the adaptive-reblocking option: the reblocked layout
+(bsa_reblock), the row gathers into it, the four stages on it and the scatter
+of O back, every step.
 ``--precision fp8`` times the FP8 (e4m3) option instead: the same stages plus
 the quantisation of the attention operands, then the e4m3 attention kernel;
 its roofline peak is the measured bf16 peak times the nominal e4m3/bf16
@@ -51,7 +54,29 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"])
-    return ap.parse_args()
+    ap.add_argument("--reblock", action="store_true")
+    args = ap.parse_args()
+    if args.reblock and args.precision != "bf16":
+        ap.error("--reblock runs the bf16 path")
+    return args
+
+
+def reblock_launches(N: int, prefix: int) -> int:
+    """Kernels bsa_reblock launches (its tree shape depends on N - prefix only):
+    init + key moment (Gram, reduction) + factor + whiten, then per level a
+    Gram, a projection and a split, plus a partial-sum pass on levels whose
+    largest group spans more than one 2048-row chunk."""
+    nv = N - prefix
+    levels = 0
+    while (128 << levels) < nv:
+        levels += 1
+    if levels == 0:
+        return 1
+    n, largest = 5, nv
+    for _ in range(levels):
+        n += 3 + (1 if largest > 2048 else 0)
+        largest -= ((largest + 127) // 128 // 2) * 128
+    return n
 
 
 def load_peaks():
@@ -178,12 +203,14 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle
 
-def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False):
+def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False, reblock=False):
     """The fp64 oracle as it stands, on whole heads, until ~budget_s of CPU work
-    (the FP8 oracle for ``fp8``)."""
+    (the FP8 oracle for ``fp8``, the reblocking oracle for ``reblock``)."""
     import oracle as orc
     from oracle import bsa_oracle_fp8 as orc8
-    head_fn = orc8.forward_head_fp8 if fp8 else orc.forward_head
+    from oracle import bsa_oracle_reblock as orcr
+    head_fn = orc8.forward_head_fp8 if fp8 else (orcr.forward_head_reblock if reblock
+                                                  else orc.forward_head)
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
@@ -202,7 +229,7 @@ def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False):
     flops = 4 * 128 * pairs
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{heads} of {cfg['H']} heads of the workload, whole "
-                      f"{'FP8 ' if fp8 else ''}path per head "
+                      f"{'FP8 ' if fp8 else ''}{'reblocked ' if reblock else ''}path per head "
                       f"(numpy fp64, BLAS threads = {cores}); {dt:.1f} s, "
                       f"{dt / heads:.2f} s/head"}, dt / heads
 
@@ -303,9 +330,18 @@ def main():
     O = torch.empty_like(Q)
     stream = torch.cuda.current_stream(dev)
     fp8 = args.precision == "fp8"
+    rbl = args.reblock
     if fp8:
         ops_buf, ops, _ = bsa.fp8_operands(p, dev)
-    names = ["pool", "summarize", "select"] + (["quantize"] if fp8 else []) + ["attend"]
+    if rbl:
+        perm = torch.empty(B, H, N, dtype=torch.int32, device=dev)
+        rb_ws = torch.empty(max(256, bsa.bsa_reblock_workspace_bytes(p)), dtype=torch.uint8,
+                            device=dev)
+        Qa, Ka, Va, Oa = (torch.empty_like(Q) for _ in range(4))
+    else:
+        Qa, Ka, Va, Oa = Q, K, V, O
+    names = (["reblock", "permute"] if rbl else []) + ["pool", "summarize", "select"] + \
+        (["quantize"] if fp8 else []) + ["attend"] + (["unpermute"] if rbl else [])
     nev = len(names) + 1
 
     def step(ev=None):
@@ -315,9 +351,14 @@ def main():
             if ev:
                 next(marks).record(stream)
         mark()
-        bsa.bsa_pool(p, Q, buf["qpool"], buf["anchor"], stream)
+        if rbl:
+            bsa.bsa_reblock(p, Q, K, perm, rb_ws, stream)
+            mark()
+            bsa.bsa_permute(p, Q, K, V, perm, Qa, Ka, Va, stream)
+            mark()
+        bsa.bsa_pool(p, Qa, buf["qpool"], buf["anchor"], stream)
         mark()
-        bsa.bsa_summarize(p, K, V, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"],
+        bsa.bsa_summarize(p, Ka, Va, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"],
                           buf["bias"], stream)
         mark()
         bsa.bsa_select(p, buf["qpool"], buf["kpool"], buf["idx"], buf["cnt"], stream)
@@ -327,9 +368,12 @@ def main():
             mark()
             bsa.bsa_attend_fp8(p, ops, buf["idx"], buf["cnt"], buf["bias"], O, None, stream)
         else:
-            bsa.bsa_attend(p, Q, K, V, buf["idx"], buf["cnt"], buf["ksum"], buf["vsum"],
-                           buf["bias"], O, None, stream)
+            bsa.bsa_attend(p, Qa, Ka, Va, buf["idx"], buf["cnt"], buf["ksum"], buf["vsum"],
+                           buf["bias"], Oa, None, stream)
         mark()
+        if rbl:
+            bsa.bsa_unpermute(p, Oa, None, perm, O, None, stream)
+            mark()
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -367,18 +411,26 @@ def main():
 
     # end to end through the C ABI from pinned host buffers
     e2e = None
-    if not args.no_e2e and fp8:
-        # the public FP8 call from pinned host buffers: copies in, forward_fp8,
-        # O copied back, all inside the timed region
+    if not args.no_e2e and (fp8 or rbl):
+        # the public call from pinned host buffers: copies in, forward_fp8 /
+        # forward_reblock, O copied back, all inside the timed region
         hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
         hO = torch.empty_like(hQ).pin_memory()
-        ws8 = torch.empty(bsa.bsa_forward_fp8_workspace_bytes(p), dtype=torch.uint8, device=dev)
+        if fp8:
+            ws8 = torch.empty(bsa.bsa_forward_fp8_workspace_bytes(p), dtype=torch.uint8,
+                              device=dev)
+            fwd, fwd_name = bsa.bsa_forward_fp8, "bsa_forward_fp8"
+        else:
+            del Qa, Ka, Va, Oa, rb_ws
+            ws8 = torch.empty(bsa.bsa_forward_reblock_workspace_bytes(p), dtype=torch.uint8,
+                              device=dev)
+            fwd, fwd_name = bsa.bsa_forward_reblock, "bsa_forward_reblock"
 
         def e2e_call():
             Q.copy_(hQ, non_blocking=True)
             K.copy_(hK, non_blocking=True)
             V.copy_(hV, non_blocking=True)
-            bsa.bsa_forward_fp8(p, Q, K, V, O, None, ws8, stream)
+            fwd(p, Q, K, V, O, None, ws8, stream)
             hO.copy_(O, non_blocking=True)
         for _ in range(2):
             e2e_call()
@@ -396,7 +448,7 @@ def main():
                "unit": "TFLOP/s", "ms_per_call": e_ms / args.e2e_steps,
                "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                "d2h_bytes_per_step": O.numel() * O.element_size(),
-               "path": "bsa_forward_fp8 with pinned-host copies in and out (one stream)"}
+               "path": f"{fwd_name} with pinned-host copies in and out (one stream)"}
         del hQ, hK, hV, hO, ws8
     elif not args.no_e2e:
         hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
@@ -422,11 +474,12 @@ def main():
         del hQ, hK, hV, hO
 
     peaks, peak_src = load_peaks()
-    attend_ms = stage_ms[-1]
+    attend_ms = stage_ms[names.index("attend")]
     attend_tflops = flops_step / (attend_ms / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"]) * (2.0 if fp8 else 1.0)
     pool_bytes = stage_bytes(B, H, N, nb, bsa.bsa_select_capacity(p))
-    pool_gbs = pool_bytes / ((stage_ms[0] + stage_ms[1]) / 1e3) / 1e9
+    pool_gbs = pool_bytes / ((stage_ms[names.index("pool")] + stage_ms[names.index("summarize")])
+                             / 1e3) / 1e9
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -434,7 +487,7 @@ def main():
         Qh = [Q[0, h].double().cpu().numpy() for h in hh]
         Kh = [K[0, h].double().cpu().numpy() for h in hh]
         Vh = [V[0, h].double().cpu().numpy() for h in hh]
-        cpu, _ = time_oracle(Qh, Kh, Vh, cfg, fp8=fp8)
+        cpu, _ = time_oracle(Qh, Kh, Vh, cfg, fp8=fp8, reblock=rbl)
 
     if rank == 0:
         line = {
@@ -443,7 +496,9 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3" if fp8 else "bf16",
             "data": "synthetic (seeded per-block-offset bf16 Q/K/V of the H3 768p-5s shape)",
-            "config": config_block(cfg, parallelism=f"{world} independent calls (one per GPU)"),
+            "config": config_block(cfg, parallelism=f"{world} independent calls (one per GPU)",
+                                   **({"layout": "adaptive reblocking (q_reuse_k)"} if rbl
+                                      else {})),
             "ms_per_call": ms_per_step,
             "effective_tflop_per_call": flops_step / 1e12,
             "stages_ms": dict(zip(names, stage_ms)),
@@ -459,7 +514,8 @@ def main():
                              "bytes_per_call": pool_bytes},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": (11 if fp8 else 5) * args.steps,
+            "gpu_launches": ((11 if fp8 else 5) + (reblock_launches(N, prefix) + 2 if rbl else 0))
+                            * args.steps,
             "clocks": clock_info,
             "context": {"pages_rtx_pro_6000_sparse_ms": 30.7 if cfg["N"] == 37_740 else None},
         }

@@ -243,6 +243,7 @@ size_t reblock_carve(const Shape& s, const bsa::ReblockPlan& plan, uint8_t* base
   uint8_t* part = take(bh * plan.max_partials * 128 * 128 * 4);
   uint8_t* psum = take(bh * plan.max_partials * 128 * 4);
   uint8_t* vdir = take(bh * (static_cast<size_t>(1) << plan.levels) * 128 * 4);
+  uint8_t* moment = take(bh * 128 * 128 * 4);
   uint8_t* r_hi = take(bh * 128 * 128 * 2);
   uint8_t* r_lo = take(bh * 128 * 128 * 2);
   uint8_t* u = take(bh * nv * 128 * 2);
@@ -252,6 +253,7 @@ size_t reblock_carve(const Shape& s, const bsa::ReblockPlan& plan, uint8_t* base
     w->part = reinterpret_cast<float*>(part);
     w->psum = reinterpret_cast<float*>(psum);
     w->vdir = reinterpret_cast<float*>(vdir);
+    w->moment = reinterpret_cast<float*>(moment);
     w->r_hi = reinterpret_cast<__nv_bfloat16*>(r_hi);
     w->r_lo = reinterpret_cast<__nv_bfloat16*>(r_lo);
     w->u = reinterpret_cast<__nv_bfloat16*>(u);

@@ -76,6 +76,7 @@ struct ReblockBuffers {
   float* part;            // [BH, max_partials, 128, 128]
   float* psum;            // [BH, max_partials, 128]
   float* vdir;            // [BH, 2^levels, 128]
+  float* moment;          // [BH, 128, 128] key second moment
   __nv_bfloat16* r_hi;    // [BH, 128, 128]
   __nv_bfloat16* r_lo;    // [BH, 128, 128]
   __nv_bfloat16* u;       // [BH, nv, 128]

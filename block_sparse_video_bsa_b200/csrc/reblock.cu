@@ -122,17 +122,20 @@ struct GramArgs {
   int* dev_status;
 };
 
+constexpr int kStages = 3;   // Gram tiles in flight (cp.async ring)
+
 struct GramSmem {
-  uint64_t done[2];
+  uint64_t done[kStages];
   uint32_t tmem_base;
   int abort_flag;
   float c[128], v[128], red[4];
+  int32_t rows[kChunkTok];   // group mode: u row of each position of the chunk
 };
 
 template <bool kGroup>
 __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
   extern __shared__ __align__(1024) uint8_t sm[];
-  GramSmem* ctl = reinterpret_cast<GramSmem*>(sm + 2 * kTile);
+  GramSmem* ctl = reinterpret_cast<GramSmem*>(sm + kStages * kTile);
   const int tid = threadIdx.x;
   const size_t bh = blockIdx.y;
   int slot = 0, chunk = blockIdx.x, p0, p1;
@@ -153,14 +156,17 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
   }
 
   if (tid == 0) {
-    mbar_init(&ctl->done[0], 1);
-    mbar_init(&ctl->done[1], 1);
+    for (int i = 0; i < kStages; ++i) mbar_init(&ctl->done[i], 1);
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
   if (tid < 32) {
     tmem_alloc(&ctl->tmem_base, 128);
     tmem_relinquish();
+  }
+  if constexpr (kGroup) {   // the chunk's rows of u, read once
+    for (int i = tid; i < p1 - p0; i += 128)
+      ctl->rows[i] = __ldg(a.perm + bh * a.N + a.prefix + p0 + i) - a.prefix;
   }
   tc_fence_before();
   __syncthreads();
@@ -171,36 +177,67 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
 
   auto row_ptr = [&](int pos) -> const __nv_bfloat16* {
     if constexpr (kGroup) {
-      const int orig = __ldg(a.perm + bh * a.N + a.prefix + pos);
-      return a.X + (bh * a.nv + (orig - a.prefix)) * kDim;
+      return a.X + (bh * a.nv + ctl->rows[pos - p0]) * kDim;
     } else {
       return a.X + (bh * a.N + a.prefix + pos) * kDim;
     }
   };
 
   const int ntile = (p1 - p0 + kBlock - 1) / kBlock;
+  const int c16 = tid & 15;
+  // Tiles stream through a ring of kStages buffers with cp.async (16 bytes
+  // per copy, rows ps*8 + tid/16), two tiles ahead of the MMA: each thread's
+  // copies of a tile form one commit group (empty past the last tile, so the
+  // group count stays uniform).  Rows past the chunk are zero-filled.
+  auto issue_tile = [&](int it) {
+    if (it < ntile) {
+      const int base = p0 + it * kBlock;
+      const int nrow = min(kBlock, p1 - base);
+      uint8_t* buf = sm + (it % kStages) * kTile;
+#pragma unroll
+      for (int ps = 0; ps < 16; ++ps) {
+        const int r = ps * 8 + (tid >> 4);
+        const bool valid = r < nrow;
+        cp_async16(buf + swz(r, c16),
+                   reinterpret_cast<const uint4*>(row_ptr(valid ? base + r : p0)) + c16,
+                   valid ? 16u : 0u);
+      }
+    }
+    cp_async_commit();
+  };
+  issue_tile(0);
+  issue_tile(1);
   float colsum = 0.f;
   bool ok = true;
   for (int it = 0; it < ntile && ok; ++it) {
-    const int b = it & 1;
-    if (it >= 2 && !mbar_wait(&ctl->done[b], ((it - 2) >> 1) & 1, wc)) { ok = false; break; }
-    uint8_t* buf = sm + b * kTile;
-    const int base = p0 + it * kBlock;
-    const int nrow = min(kBlock, p1 - base);
-#pragma unroll 4
-    for (int ps = 0; ps < 16; ++ps) {
-      const int r = ps * 8 + (tid >> 4), c16 = tid & 15;
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (r < nrow) w = ld_stream_v4(reinterpret_cast<const uint4*>(row_ptr(base + r)) + c16);
-      *reinterpret_cast<uint4*>(buf + swz(r, c16)) = w;
+    // buffer (it + 2) % kStages last held tile it - 1: its MMAs must be done
+    // and every thread past its column sums before it is refilled
+    if (it >= 1) {
+      __syncthreads();
+      if (!mbar_wait(&ctl->done[(it - 1) % kStages], ((it - 1) / kStages) & 1, wc)) {
+        ok = false;
+        break;
+      }
     }
+    issue_tile(it + 2);
+    cp_async_wait<2>();   // this thread's copies of tile it have landed
     fence_proxy_async_smem();
     __syncthreads();
-    if constexpr (kGroup) {   // column tid of the tile's rows
-      const int c16 = tid >> 3, e = tid & 7;
-      for (int r = 0; r < nrow; ++r)
-        colsum += __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16*>(buf + swz(r, c16) + 2 * e));
+    const uint8_t* buf = sm + (it % kStages) * kTile;
+    if constexpr (kGroup) {   // column tid of the tile's rows (rows past nrow are zero)
+      const int cc = tid >> 3, e = tid & 7;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll 4
+      for (int r = 0; r < kBlock; r += 4) {
+        s0 += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(buf + swz(r, cc) + 2 * e));
+        s1 += __bfloat162float(
+            *reinterpret_cast<const __nv_bfloat16*>(buf + swz(r + 1, cc) + 2 * e));
+        s2 += __bfloat162float(
+            *reinterpret_cast<const __nv_bfloat16*>(buf + swz(r + 2, cc) + 2 * e));
+        s3 += __bfloat162float(
+            *reinterpret_cast<const __nv_bfloat16*>(buf + swz(r + 3, cc) + 2 * e));
+      }
+      colsum += (s0 + s1) + (s2 + s3);
     }
     if (tid == 0) {
       tc_fence_after();
@@ -210,12 +247,13 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
         const uint64_t d = smem_desc_sw128(addr + kk * 2048, kHalf, 1024);
         mma_bf16_ss(tmem, d, d, idesc, (it > 0 || kk > 0) ? 1u : 0u);
       }
-      mma_commit(&ctl->done[b]);
+      mma_commit(&ctl->done[it % kStages]);
     }
   }
+  cp_async_wait<0>();
   // the last tile's MMAs (all earlier ones complete in order before it)
   const int last = ntile - 1;
-  if (ok && !mbar_wait(&ctl->done[last & 1], (last >> 1) & 1, wc)) ok = false;
+  if (ok && !mbar_wait(&ctl->done[last % kStages], (last / kStages) & 1, wc)) ok = false;
   ok = __syncthreads_and(ok);
   tc_fence_after();
 
@@ -285,9 +323,33 @@ __global__ void __launch_bounds__(128) group_kernel(const GramArgs a) {
   power_iterate(gr, n, c, v, red, a.vdir + (bh * a.slots + slot) * kDim);
 }
 
+// Fixed-order sum of the key-moment chunk partials: row blockIdx.x of M.
+__global__ void __launch_bounds__(128) moment_reduce_kernel(const float* __restrict__ part,
+                                                            int nchunk, float* __restrict__ M) {
+  const int i = blockIdx.x, j = threadIdx.x;
+  const size_t bh = blockIdx.y;
+  float s = 0.f;
+  for (int ch = 0; ch < nchunk; ++ch) s += part[((bh * nchunk + ch) * 128 + i) * 128 + j];
+  M[(bh * 128 + i) * 128 + j] = s;
+}
+
+// dot of rows a and b of the shared matrix over k < n, four partial sums.
+__device__ __forceinline__ double row_dot(const double* a, const double* b, int n) {
+  double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+  int k = 0;
+  for (; k + 4 <= n; k += 4) {
+    s0 = fma(a[k], b[k], s0);
+    s1 = fma(a[k + 1], b[k + 1], s1);
+    s2 = fma(a[k + 2], b[k + 2], s2);
+    s3 = fma(a[k + 3], b[k + 3], s3);
+  }
+  for (; k < n; ++k) s0 = fma(a[k], b[k], s0);
+  return (s0 + s1) + (s2 + s3);
+}
+
 // Cholesky of the key second moment (fp64, in shared memory, lower triangle
 // in place) and R = L^T split into bf16 hi + lo.
-__global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ part, int nchunk,
+__global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ Mg,
                                                      __nv_bfloat16* __restrict__ r_hi,
                                                      __nv_bfloat16* __restrict__ r_lo) {
   extern __shared__ double M[];   // [128][129]
@@ -295,12 +357,7 @@ __global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ p
   const int tid = threadIdx.x;
   const size_t bh = blockIdx.x;
   constexpr int ld = 129;
-  for (int i = 0; i < 128; ++i) {   // column tid of row i (coalesced)
-    double s = 0.0;
-    for (int ch = 0; ch < nchunk; ++ch)
-      s += part[((bh * nchunk + ch) * 128 + i) * 128 + tid];
-    M[i * ld + tid] = s;
-  }
+  for (int i = 0; i < 128; ++i) M[i * ld + tid] = Mg[(bh * 128 + i) * 128 + tid];
   __syncthreads();
   red[tid] = M[tid * ld + tid];
   __syncthreads();
@@ -315,14 +372,12 @@ __global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ p
   __syncthreads();
   for (int j = 0; j < 128; ++j) {
     if (tid == 0) {
-      double s = M[j * ld + j];
-      for (int k = 0; k < j; ++k) s -= M[j * ld + k] * M[j * ld + k];
+      const double s = M[j * ld + j] - row_dot(M + j * ld, M + j * ld, j);
       M[j * ld + j] = sqrt(s > 0.0 ? s : 1e-300);
     }
     __syncthreads();
     if (tid > j) {
-      double s = M[tid * ld + j];
-      for (int k = 0; k < j; ++k) s -= M[tid * ld + k] * M[j * ld + k];
+      const double s = M[tid * ld + j] - row_dot(M + tid * ld, M + j * ld, j);
       M[tid * ld + j] = s / M[j * ld + j];
     }
     __syncthreads();
@@ -456,24 +511,34 @@ __global__ void __launch_bounds__(256) project_kernel(const __nv_bfloat16* __res
   float vv[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) vv[e] = v[8 * c16 + e];
-  // every half-warp runs the same number of iterations (the shuffles below
-  // span the whole warp); the tail masks the load instead
-  for (int base = p0; base < p1; base += 16) {
-    const int pos = base + (tid >> 4);
-    const bool valid = pos < p1;
-    uint4 w = make_uint4(0, 0, 0, 0);
-    if (valid) {
-      const int orig = __ldg(perm + bh * N + prefix + pos);
-      w = ld_stream_v4(reinterpret_cast<const uint4*>(u + (bh * nv + (orig - prefix)) * kDim) +
-                       c16);
+  // 4 positions per 16-lane group in flight; every half-warp runs the same
+  // number of iterations (the shuffles below span the whole warp) and the
+  // tail masks the loads instead
+  constexpr int kPer = 4;
+  for (int base = p0; base < p1; base += 16 * kPer) {
+    int orig[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int pos = base + (tid >> 4) + 16 * k;
+      orig[k] = pos < p1 ? __ldg(perm + bh * N + prefix + pos) : -1;
     }
-    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&w);
-    float s = 0.f;
+    uint4 w[kPer];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) s = fmaf(__bfloat162float(h[e]), vv[e], s);
+    for (int k = 0; k < kPer; ++k)
+      w[k] = orig[k] >= 0 ? ld_stream_v4(reinterpret_cast<const uint4*>(
+                                             u + (bh * nv + (orig[k] - prefix)) * kDim) + c16)
+                          : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (valid && c16 == 0) keys[bh * nv + pos] = orderable_key(s);
+    for (int k = 0; k < kPer; ++k) {
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&w[k]);
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s = fmaf(__bfloat162float(h[e]), vv[e], s);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      const int pos = base + (tid >> 4) + 16 * k;
+      if (orig[k] >= 0 && c16 == 0) keys[bh * nv + pos] = orderable_key(s);
+    }
   }
 }
 
@@ -524,19 +589,26 @@ __global__ void __launch_bounds__(512) split_kernel(const uint32_t* __restrict__
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += 512) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < g.count; i += 512) {
-      const uint32_t x = __ldg(k + i);
-      if ((x & mask) == prefix_bits) atomicAdd(&hist[(x >> shift) & 255u], 1);
+    for (int i0 = 0; i0 < g.count; i0 += 4 * 512) {   // four keys per thread in flight
+      uint32_t x[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = i0 + q * 512 + tid;
+        x[q] = i < g.count ? __ldg(k + i) : 0u;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (i0 + q * 512 + tid < g.count && (x[q] & mask) == prefix_bits)
+          atomicAdd(&hist[(x[q] >> shift) & 255u], 1);
     }
     __syncthreads();
-    if (tid == 0) {
-      int run = 0, d = 0;
-      for (d = 0; d < 255; ++d) {
-        if (run + hist[d] >= want) break;
-        run += hist[d];
+    {   // the digit d with (count below d) < want <= (count through d)
+      const int h = tid < 256 ? hist[tid] : 0;
+      const int below = block_scan(h, wsum, &sh[2]);
+      if (tid < 256 && below < want && want <= below + h) {
+        sh[0] = tid;
+        sh[1] = want - below;
       }
-      sh[0] = d;
-      sh[1] = want - run;
     }
     __syncthreads();
     prefix_bits |= static_cast<uint32_t>(sh[0]) << shift;
@@ -549,10 +621,12 @@ __global__ void __launch_bounds__(512) split_kernel(const uint32_t* __restrict__
   int left_run = 0, eq_run = 0;
   const int32_t* pin = perm_in + bh * N + prefix + g.start;
   int32_t* pout = perm_out + bh * N + prefix + g.start;
+  uint32_t x_next = tid < g.count ? __ldg(k + tid) : 0xffffffffu;
   for (int base = 0; base < g.count; base += 512) {
     const int i = base + tid;
     const bool valid = i < g.count;
-    const uint32_t x = valid ? __ldg(k + i) : 0xffffffffu;
+    const uint32_t x = x_next;   // loaded one round ahead
+    x_next = (i + 512 < g.count) ? __ldg(k + i + 512) : 0xffffffffu;
     const int eq = (valid && x == T) ? 1 : 0;
     int eq_tot;
     const int eq_before = eq_run + block_scan(eq, wsum, &sh[2]);
@@ -642,7 +716,7 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
   const int BH = s.B * s.H;
   const int nv = plan.nv;
   // Gram kernels: two 32 KB tiles + control; factor: 128 x 129 doubles.
-  const size_t gram_smem = 2 * kTile + sizeof(GramSmem) + 1024;
+  const size_t gram_smem = kStages * kTile + sizeof(GramSmem) + 1024;
   const size_t whiten_smem = 3 * kTile + sizeof(WhitenSmem) + 1024;
   const size_t factor_smem = 128 * 129 * sizeof(double);
   static bool attr[64] = {false};
@@ -681,7 +755,8 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
   ga.slots = 1;
   ga.max_chunks = plan.moment_chunks;
   gram_kernel<false><<<dim3(plan.moment_chunks, BH), 128, gram_smem, st>>>(ga);
-  factor_kernel<<<BH, 128, factor_smem, st>>>(w.part, plan.moment_chunks, w.r_hi, w.r_lo);
+  moment_reduce_kernel<<<dim3(128, BH), 128, 0, st>>>(w.part, plan.moment_chunks, w.moment);
+  factor_kernel<<<BH, 128, factor_smem, st>>>(w.moment, w.r_hi, w.r_lo);
   whiten_kernel<<<dim3((nv + kBlock - 1) / kBlock, BH), 128, whiten_smem, st>>>(
       maps.q, maps.r_hi, maps.r_lo, s.prefix, nv, w.u, s.dev_status);
   (void)Q;
