@@ -22,7 +22,14 @@ namespace bsa {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kPadT = 128 + 16;   // transpose tile row (bytes), padded against bank conflicts
+
+// Byte (r, c) of the 128 x 128-byte transpose tile: 16-byte chunks of a row
+// are XOR-swizzled by r / 16, so the column reads of the transpose (16 rows
+// r0..r0+15 of 4 adjacent columns per 4 lanes, 8 row groups per warp) touch 8
+// different banks.
+__device__ __forceinline__ int tswz(int r, int c) {
+  return r * 128 + ((((c >> 4) ^ (r >> 4)) & 7) << 4) + (c & 15);
+}
 
 template <bool kTranspose>
 __global__ void __launch_bounds__(kThreads) quant_kernel(const __nv_bfloat16* __restrict__ X,
@@ -30,7 +37,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __nv_bfloat16* __
                                                          uint8_t* __restrict__ codes,
                                                          float* __restrict__ scale) {
   __shared__ float red[kThreads / 32];
-  __shared__ __align__(16) uint8_t tile[kTranspose ? 128 * kPadT : 16];
+  __shared__ __align__(16) uint8_t tile[kTranspose ? 128 * 128 : 16];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = blockIdx.x;
   const size_t bh = blockIdx.y;
@@ -73,7 +80,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __nv_bfloat16* __
                               __fmul_rn(x[ps][6], ratio), __fmul_rn(x[ps][7], ratio));
     if (r >= nrows) w0 = w1 = 0u;
     if constexpr (kTranspose) {
-      *reinterpret_cast<uint2*>(tile + r * kPadT + 8 * c8) = make_uint2(w0, w1);
+      *reinterpret_cast<uint2*>(tile + tswz(r, 8 * c8)) = make_uint2(w0, w1);
     } else if (r < nrows) {
       *reinterpret_cast<uint2*>(codes + (bh * rows + r0 + r) * kDim + 8 * c8) = make_uint2(w0, w1);
     }
@@ -90,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __nv_bfloat16* __
         uint32_t v = 0;
 #pragma unroll
         for (int b = 0; b < 4; ++b)
-          v |= static_cast<uint32_t>(tile[(rc * 16 + q * 4 + b) * kPadT + dim]) << (8 * b);
+          v |= static_cast<uint32_t>(tile[tswz(rc * 16 + q * 4 + b, dim)]) << (8 * b);
         w[q] = v;
       }
       *reinterpret_cast<uint4*>(out + dim * kBlock + rc * 16) = make_uint4(w[0], w[1], w[2], w[3]);

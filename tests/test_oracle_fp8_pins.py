@@ -154,3 +154,33 @@ def test_output_bound_covers_simulated_e4m3_numerators():
         sq_err += float((err ** 2).sum())
     # the squared error over all elements stays within the variance model
     assert sq_err <= var.sum(), (sq_err, var.sum())
+
+
+def test_output_bound_needs_its_subnormal_term():
+    # Peaked logits: most numerators p * r fall below 2^-6, where e4m3 is
+    # subnormal and its error is absolute (2^-10), not relative.  The full
+    # bound must hold on the brute-force simulation; its relative part alone
+    # must not (so the absolute term is load-bearing).
+    rng = np.random.default_rng(6)
+    N, d, top_k = 512, 8, 4
+    Q = rng.standard_normal((N, d)) * 4.0
+    K = rng.standard_normal((N, d)) * 4.0
+    V = rng.standard_normal((N, d))
+    r8 = f8.forward_head_fp8(Q, K, V, top_k, 0)
+    bound = f8.fp8_output_bound(r8["Qd"], r8["Kd"], r8["Vd"], r8["lists"], r8["KSd"], r8["VSd"],
+                                r8["bias"], r8["v_scale"], r8["vs_scale"], 0)
+    s_ref = max(r8["v_scale"].max(), r8["vs_scale"].max())
+    rel_only_violated = False
+    for i, (a, b) in enumerate(orc.block_bounds(N)):
+        E = [int(j) for j in r8["lists"][i]]
+        tok = np.concatenate([np.arange(*orc.block_bounds(N)[j]) for j in E])
+        logits = r8["Qd"][a:b] @ r8["Kd"][tok].T / np.sqrt(d)           # every block listed
+        r = r8["v_scale"][tok // 128] / s_ref
+        p = np.exp(logits - logits.max(axis=1, keepdims=True))
+        l = p.sum(axis=1, keepdims=True)
+        O_sim = s_ref * (f8.round_e4m3(p * r[None, :]) @ r8["v_codes"][tok]) / l
+        err = np.abs(O_sim - r8["O"][a:b])
+        assert (err <= bound[a:b] + 1e-12).all()
+        rel_only = (2.0 ** -4 * p / l) @ np.abs(r8["Vd"][tok])
+        rel_only_violated |= bool((err > rel_only + 1e-12).any())
+    assert rel_only_violated
