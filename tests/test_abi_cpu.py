@@ -87,3 +87,57 @@ def test_density_to_topk_rounds_up():
     assert [bsa.topk_from_density(r, 133_644) for r in (0.1, 0.2, 0.3)] == [105, 209, 314]
     assert bsa.topk_from_density(0.3, 128_000) == 300
     assert bsa.topk_from_density(0.001, 2048) == 1
+
+
+def test_option_sizes():
+    # reblocking scratch and the FP8 operand set follow the documented layouts
+    p = _p()
+    bh, N, nb = 56, 37_740, 295
+    ops = bsa.bsa_fp8_operands_bytes(p)
+    codes = bh * N * 128 * 2 + bh * nb * 128 * 128 + bh * nb * 128 + bh * 3 * 128 * 128
+    scales = (3 * bh * nb + 2 * bh * 3 + bh) * 4
+    assert codes + scales <= ops <= codes + scales + 11 * 256
+    assert bsa.bsa_forward_fp8_workspace_bytes(p) == bsa.bsa_workspace_bytes(p) + ops
+    rb = bsa.bsa_reblock_workspace_bytes(p)
+    assert rb >= bh * (N - 0) * 128 * 2 + bh * N * 4      # bf16 whitened queries + a permutation
+    frb = bsa.bsa_forward_reblock_workspace_bytes(p)
+    assert frb >= rb + bsa.bsa_workspace_bytes(p) + 4 * bh * N * 256
+    for f in (bsa.bsa_fp8_operands_bytes, bsa.bsa_reblock_workspace_bytes,
+              bsa.bsa_forward_reblock_workspace_bytes, bsa.bsa_forward_fp8_workspace_bytes):
+        assert f(_p(top_k=0)) == 0
+
+
+def test_option_arguments_rejected_before_launch():
+    L = bsa.lib()
+    p = _p()
+    P = ctypes.byref(p)
+    a = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    # reblocking
+    assert L.bsa_reblock(P, a, a, None, a, 1 << 40, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_reblock(P, a, a, a, a, 16, None) == bsa.BSA_ERR_INVALID      # scratch too small
+    assert L.bsa_reblock(P, odd, a, a, a, 1 << 40, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_permute(P, a, a, a, None, a, a, a, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_unpermute(P, a, None, a, a, a, None) == bsa.BSA_ERR_INVALID   # lse without lsep
+    assert L.bsa_forward_reblock(P, a, a, a, a, None, a, 16, None) == bsa.BSA_ERR_INVALID
+    # FP8
+    ops = bsa.bsa_fp8_operands()
+    assert L.bsa_quantize_fp8(P, a, a, a, a, a, ctypes.byref(ops), None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_attend_fp8(P, ctypes.byref(ops), a, a, a, a, None, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_fp8_operands_carve(P, a, 16, ctypes.byref(ops)) == bsa.BSA_ERR_INVALID
+    assert L.bsa_fp8_operands_carve(P, odd, 1 << 40, ctypes.byref(ops)) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_forward_fp8(P, a, a, a, a, None, a, 16, None) == bsa.BSA_ERR_INVALID
+
+
+def test_fp8_operands_carve_follows_the_field_order():
+    # carving needs no device: it only computes pointers into the caller's buffer
+    L = bsa.lib()
+    p = _p(N=1000, H=2)
+    n = bsa.bsa_fp8_operands_bytes(p)
+    base = 1 << 32
+    ops = bsa.bsa_fp8_operands()
+    assert L.bsa_fp8_operands_carve(ctypes.byref(p), ctypes.c_void_p(base), n,
+                                    ctypes.byref(ops)) == bsa.BSA_OK
+    ptrs = [getattr(ops, f) for f, _ in bsa.bsa_fp8_operands._fields_]
+    assert ptrs[0] == base and all(b > a for a, b in zip(ptrs, ptrs[1:]))
+    assert all(x % 256 == 0 for x in ptrs) and ptrs[-1] < base + n
