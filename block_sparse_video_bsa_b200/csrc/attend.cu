@@ -376,13 +376,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&ctl->bias_empty[s][v & 1]);
         mul = make_float2(1.f, 1.f);
       }
+      // row max: 8 independent chains of three-input maxes (64 instructions)
       float mp[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mp[k] = x[k];
+      for (int k = 0; k < 8; ++k) mp[k] = fmaxf(x[k], x[k + 8]);
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * mul.x;
+      for (int c = 16; c < 128; c += 16) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mp[k] = fmax3(mp[k], x[c + k], x[c + 8 + k]);
+      }
+      const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
+                             fmaxf(mp[6], mp[7])) * mul.x;
       const bool need = mx > m_run + kRescaleThreshold;
       const float m_new = need ? mx : m_run;
       const float alpha = need ? fast_exp2(m_run - m_new) : 1.0f;

@@ -62,6 +62,14 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input max; a NaN operand is
+// ignored, as with fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Per-warpgroup register budget (all four warps of a warpgroup execute it;
 // the budgets of all warpgroups must add up to the launch allocation).
 template <uint32_t kRegs>
