@@ -91,12 +91,15 @@ __device__ __forceinline__ void power_iterate(const float (&g)[128], float n, fl
   v[i] = 0.08838834764831845f;   // 1 / sqrt(128)
   __syncthreads();
   for (int it = 0; it < kPowerIters; ++it) {
-    float cv = 0.f, w = 0.f;
+    // four independent partial sums per dot product (fixed order)
+    float cv4[4] = {0.f, 0.f, 0.f, 0.f}, w4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll   // fully: g[] stays in registers
     for (int j = 0; j < 128; ++j) {
-      cv = fmaf(c[j], v[j], cv);
-      w = fmaf(g[j], v[j], w);
+      cv4[j & 3] = fmaf(c[j], v[j], cv4[j & 3]);
+      w4[j & 3] = fmaf(g[j], v[j], w4[j & 3]);
     }
+    const float cv = (cv4[0] + cv4[1]) + (cv4[2] + cv4[3]);
+    float w = (w4[0] + w4[1]) + (w4[2] + w4[3]);
     w = fmaf(-n * c[i], cv, w);
     float s = w * w;
 #pragma unroll
