@@ -141,3 +141,34 @@ def test_fp8_operands_carve_follows_the_field_order():
     ptrs = [getattr(ops, f) for f, _ in bsa.bsa_fp8_operands._fields_]
     assert ptrs[0] == base and all(b > a for a, b in zip(ptrs, ptrs[1:]))
     assert all(x % 256 == 0 for x in ptrs) and ptrs[-1] < base + n
+
+
+def _reblock_scratch(B, H, N, prefix):
+    """Bytes of the reblocking scratch from the tree's shape (independent
+    replica of the plan: levels, chunk counts of the largest group, partial
+    slots), each piece rounded to 256 bytes."""
+    r256 = lambda x: (x + 255) // 256 * 256
+    nv, bh = N - prefix, B * H
+    levels = 0
+    while (128 << levels) < nv:
+        levels += 1
+    moment_chunks = -(-nv // 2048)
+    maxp, largest = 1, nv
+    for l in range(levels):
+        chunks = -(-largest // 2048)
+        if chunks > 1:
+            maxp = max(maxp, (1 << l) * chunks)
+        largest -= (-(-largest // 128) // 2) * 128
+    maxp = max(maxp, moment_chunks)
+    return sum(r256(x) for x in (bh * N * 4, bh * maxp * 128 * 128 * 4, bh * maxp * 128 * 4,
+                                 bh * (1 << levels) * 128 * 4, bh * 128 * 128 * 4,
+                                 bh * 128 * 128 * 2, bh * 128 * 128 * 2, bh * nv * 128 * 2,
+                                 bh * nv * 4))
+
+
+@pytest.mark.parametrize("B,H,N,prefix", [(1, 56, 37_740, 0), (1, 56, 133_644, 0),
+                                          (1, 56, 103_996, 512), (2, 3, 4100, 0), (1, 1, 129, 0),
+                                          (1, 1, 128, 0), (1, 2, 2049, 0), (1, 1, 1, 0)])
+def test_reblock_scratch_follows_the_tree_shape(B, H, N, prefix):
+    p = bsa.params(B, H, N, 1, prefix)
+    assert bsa.bsa_reblock_workspace_bytes(p) == _reblock_scratch(B, H, N, prefix)
