@@ -19,9 +19,11 @@ READINGS of this project:
   video query block i the scores S[i, j] over the video key blocks
   j in [pb, nb) have mean mu_i and population standard deviation sigma_i
   (divided by nbv); block j is kept when S[i, j] - mu_i >= tau * sigma_i.
-* T-b (no contrast).  With ">=", a row whose scores are all equal
-  (sigma_i = 0) keeps every video block: with nothing to rank, the row is
-  read exactly.
+* T-b (no contrast).  A row whose scores are all equal (sigma_i = 0, where
+  ">=" keeps everything) keeps every video block: with nothing to rank, the
+  row is read exactly.  It is decided by comparing the row's largest and
+  smallest score, which rounding cannot disturb (a rounded mean of equal
+  values can be off by one ulp, and then so is every deviation).
 * T-c (floor).  A row keeps at least one block: when no block reaches the
   threshold (possible only for tau > 0 and few blocks, since the largest
   z-score of n values is at most sqrt(n - 1)), it keeps its top-scoring block,
@@ -54,7 +56,8 @@ def select_blocks_threshold(S: np.ndarray, tau: float, prefix_blocks: int):
     """Exact-branch block list E_i for every query block i (ascending).
 
     Video query block i >= pb: the video key blocks whose score is at least
-    tau standard deviations above the row's mean (T-a, T-b), or the single
+    tau standard deviations above the row's mean (T-a), all of them when the
+    row's scores are all equal (T-b), or else the single
     top-scoring block if none is (T-c); the pb prefix blocks in front (T-d).
     Dense-prefix query block i < pb: all nb blocks.
     """
@@ -68,7 +71,10 @@ def select_blocks_threshold(S: np.ndarray, tau: float, prefix_blocks: int):
             continue
         row = S[i, cand]
         mu, margin = row_threshold(row, tau)
-        chosen = cand[(row - mu) >= margin]
+        if row.max() == row.min():
+            chosen = cand
+        else:
+            chosen = cand[(row - mu) >= margin]
         if chosen.size == 0:
             chosen = cand[np.lexsort((cand, -row))[:1]]
         lists.append(np.concatenate([np.arange(pb), np.sort(chosen)]).astype(np.int64))

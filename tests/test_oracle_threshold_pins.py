@@ -136,6 +136,12 @@ def test_floor_and_no_contrast():
     S = np.array([[1.0, 3.0, 3.0], [0.0, 5.0, 5.0], [7.0, 2.0, 2.0]])
     assert [list(l) for l in th.select_blocks_threshold(S, 2.0, 0)] == [[1], [1], [0]]
     assert [list(l) for l in th.select_blocks_threshold(S, 0.5, 0)] == [[1, 2], [1, 2], [0]]
+    # Equal scores whose rounded mean is off by one ulp still keep every block.
+    for x, n in ((0.1, 3), (0.7, 3), (0.2, 6), (1.0, 4)):
+        row = np.full(n, x)
+        assert (row.mean() != x) == (x != 1.0)
+        lists = th.select_blocks_threshold(np.tile(row, (n, 1)), 1.5, 0)
+        assert all(list(l) == list(range(n)) for l in lists), (x, n)
 
 
 def test_invariants_on_random_rows():
