@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload h3_768p_5s] [--top-k K] [--no-cpu-baseline] [--no-e2e]
-                    [--precision bf16|fp8] [--reblock]
+                    [--precision bf16|fp8] [--reblock] [--tau T]
 
 One step = one whole attention call (pool -> summarize -> select -> attend,
 all through the C ABI) over one batch of synthetic bf16 input of the 768p-5s
@@ -13,7 +13,11 @@ of O back, every step.
 ``--precision fp8`` times the FP8 (e4m3) option instead: the same stages plus
 the quantisation of the attention operands, then the e4m3 attention kernel;
 its roofline peak is the measured bf16 peak times the nominal e4m3/bf16
-tensor ratio (2).  The default (bf16) line is the headline.
+tensor ratio (2).  ``--tau T`` times the threshold-selection option: the
+selection keeps the key blocks at least T standard deviations above each
+row's mean score (bsa_select_threshold) and the attention runs over those
+variable-length lists (bsa_attend_lists, schedule kernels included in its
+stage time).  The default (bf16, top_k) line is the headline.
 Prints ONE JSON line on rank 0.  Multi-GPU (torchrun): every rank runs its own
 independent call on its own inputs (weak scaling, no data-path collective);
 the time is the max over ranks.
@@ -55,9 +59,12 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"])
     ap.add_argument("--reblock", action="store_true")
+    ap.add_argument("--tau", type=float, default=None)
     args = ap.parse_args()
     if args.reblock and args.precision != "bf16":
         ap.error("--reblock runs the bf16 path")
+    if args.tau is not None and (args.reblock or args.precision != "bf16"):
+        ap.error("--tau runs the bf16 path without reblocking")
     return args
 
 
@@ -203,14 +210,20 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle
 
-def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False, reblock=False):
+def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False, reblock=False,
+                tau=None):
     """The fp64 oracle as it stands, on whole heads, until ~budget_s of CPU work
-    (the FP8 oracle for ``fp8``, the reblocking oracle for ``reblock``)."""
+    (the FP8 oracle for ``fp8``, the reblocking oracle for ``reblock``, the
+    threshold oracle when ``tau`` is given)."""
     import oracle as orc
     from oracle import bsa_oracle_fp8 as orc8
     from oracle import bsa_oracle_reblock as orcr
+    from oracle import bsa_oracle_threshold as orct
     head_fn = orc8.forward_head_fp8 if fp8 else (orcr.forward_head_reblock if reblock
                                                   else orc.forward_head)
+    sel = cfg["top_k"]
+    if tau is not None:
+        head_fn, sel = orct.forward_head_threshold, tau
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
@@ -220,7 +233,7 @@ def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False, reblock=
     t0 = time.perf_counter()
     heads = 0
     for h in range(min(max_heads, len(Qh))):
-        out = head_fn(Qh[h], Kh[h], Vh[h], cfg["top_k"], cfg["prefix"], cfg["variant"])
+        out = head_fn(Qh[h], Kh[h], Vh[h], sel, cfg["prefix"], cfg["variant"])
         pairs += orc.effective_pairs(len(Qh[h]), out["lists"], cfg["prefix"] // 128)
         heads += 1
         if time.perf_counter() - t0 > budget_s:
@@ -229,7 +242,8 @@ def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False, reblock=
     flops = 4 * 128 * pairs
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{heads} of {cfg['H']} heads of the workload, whole "
-                      f"{'FP8 ' if fp8 else ''}{'reblocked ' if reblock else ''}path per head "
+                      f"{'FP8 ' if fp8 else ''}{'reblocked ' if reblock else ''}"
+                      f"{'threshold ' if tau is not None else ''}path per head "
                       f"(numpy fp64, BLAS threads = {cores}); {dt:.1f} s, "
                       f"{dt / heads:.2f} s/head"}, dt / heads
 
@@ -254,8 +268,14 @@ def run_reference(args, cfg):
     times, pairs_l = [], []
     for s in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        out = orc.forward_head(heads[0], heads[1], heads[2], cfg["top_k"], cfg["prefix"],
-                               cfg["variant"], query_blocks=qblocks)
+        if args.tau is None:
+            out = orc.forward_head(heads[0], heads[1], heads[2], cfg["top_k"], cfg["prefix"],
+                                   cfg["variant"], query_blocks=qblocks)
+        else:
+            from oracle import bsa_oracle_threshold as orct
+            out = orct.forward_head_threshold(heads[0], heads[1], heads[2], args.tau,
+                                              cfg["prefix"], cfg["variant"],
+                                              query_blocks=qblocks)
         dt = time.perf_counter() - t0
         if s >= args.warmup:
             times.append(dt)
@@ -274,7 +294,10 @@ def run_reference(args, cfg):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_block(cfg, sample=sample),
+        "data": "synthetic",
+        "config": config_block(cfg, sample=sample,
+                               **({"selection": f"threshold tau={args.tau}"}
+                                  if args.tau is not None else {})),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -331,6 +354,13 @@ def main():
     stream = torch.cuda.current_stream(dev)
     fp8 = args.precision == "fp8"
     rbl = args.reblock
+    thr = args.tau is not None
+    if thr:
+        nb0 = bsa.bsa_num_blocks(p)
+        buf["idx"] = torch.empty(B, H, nb0, bsa.bsa_threshold_capacity(p), dtype=torch.int32,
+                                 device=dev)
+        lists_ws = torch.empty(bsa.bsa_attend_lists_workspace_bytes(p), dtype=torch.uint8,
+                               device=dev)
     if fp8:
         ops_buf, ops, _ = bsa.fp8_operands(p, dev)
     if rbl:
@@ -361,12 +391,19 @@ def main():
         bsa.bsa_summarize(p, Ka, Va, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"],
                           buf["bias"], stream)
         mark()
-        bsa.bsa_select(p, buf["qpool"], buf["kpool"], buf["idx"], buf["cnt"], stream)
+        if thr:
+            bsa.bsa_select_threshold(p, args.tau, buf["qpool"], buf["kpool"], buf["idx"],
+                                     buf["cnt"], stream)
+        else:
+            bsa.bsa_select(p, buf["qpool"], buf["kpool"], buf["idx"], buf["cnt"], stream)
         mark()
         if fp8:
             bsa.bsa_quantize_fp8(p, Q, K, V, buf["ksum"], buf["vsum"], ops, stream)
             mark()
             bsa.bsa_attend_fp8(p, ops, buf["idx"], buf["cnt"], buf["bias"], O, None, stream)
+        elif thr:
+            bsa.bsa_attend_lists(p, Q, K, V, buf["idx"], buf["cnt"], buf["ksum"], buf["vsum"],
+                                 buf["bias"], O, None, lists_ws, stream)
         else:
             bsa.bsa_attend(p, Qa, Ka, Va, buf["idx"], buf["cnt"], buf["ksum"], buf["vsum"],
                            buf["bias"], Oa, None, stream)
@@ -384,6 +421,10 @@ def main():
         * 1  # all B*H heads
     flops_step = 4 * 128 * pairs
     nb = bsa.bsa_num_blocks(p)
+    mean_kept = None
+    if thr:   # video blocks kept per video query block, over all heads
+        c = buf["cnt"][:, :, prefix // 128:].double()
+        mean_kept = float((c - prefix // 128).mean())
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)]
               for _ in range(args.steps)]
@@ -411,15 +452,23 @@ def main():
 
     # end to end through the C ABI from pinned host buffers
     e2e = None
-    if not args.no_e2e and (fp8 or rbl):
+    if not args.no_e2e and (fp8 or rbl or thr):
         # the public call from pinned host buffers: copies in, forward_fp8 /
-        # forward_reblock, O copied back, all inside the timed region
+        # forward_reblock / forward_threshold, O copied back, all inside the
+        # timed region
         hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
         hO = torch.empty_like(hQ).pin_memory()
         if fp8:
             ws8 = torch.empty(bsa.bsa_forward_fp8_workspace_bytes(p), dtype=torch.uint8,
                               device=dev)
             fwd, fwd_name = bsa.bsa_forward_fp8, "bsa_forward_fp8"
+        elif thr:
+            ws8 = torch.empty(bsa.bsa_forward_threshold_workspace_bytes(p), dtype=torch.uint8,
+                              device=dev)
+
+            def fwd(p_, Q_, K_, V_, O_, lse_, ws_, st_):
+                bsa.bsa_forward_threshold(p_, args.tau, Q_, K_, V_, O_, lse_, ws_, st_)
+            fwd_name = "bsa_forward_threshold"
         else:
             del Qa, Ka, Va, Oa, rb_ws
             ws8 = torch.empty(bsa.bsa_forward_reblock_workspace_bytes(p), dtype=torch.uint8,
@@ -487,7 +536,7 @@ def main():
         Qh = [Q[0, h].double().cpu().numpy() for h in hh]
         Kh = [K[0, h].double().cpu().numpy() for h in hh]
         Vh = [V[0, h].double().cpu().numpy() for h in hh]
-        cpu, _ = time_oracle(Qh, Kh, Vh, cfg, fp8=fp8, reblock=rbl)
+        cpu, _ = time_oracle(Qh, Kh, Vh, cfg, fp8=fp8, reblock=rbl, tau=args.tau)
 
     if rank == 0:
         line = {
@@ -498,7 +547,9 @@ def main():
             "data": "synthetic (seeded per-block-offset bf16 Q/K/V of the H3 768p-5s shape)",
             "config": config_block(cfg, parallelism=f"{world} independent calls (one per GPU)",
                                    **({"layout": "adaptive reblocking (q_reuse_k)"} if rbl
-                                      else {})),
+                                      else {}),
+                                   **({"selection": f"threshold tau={args.tau}",
+                                       "mean_kept_blocks": mean_kept} if thr else {})),
             "ms_per_call": ms_per_step,
             "effective_tflop_per_call": flops_step / 1e12,
             "stages_ms": dict(zip(names, stage_ms)),
@@ -519,8 +570,8 @@ def main():
                              "bytes_per_call": pool_bytes},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": ((11 if fp8 else 5) + (reblock_launches(N, prefix) + 2 if rbl else 0))
-                            * args.steps,
+            "gpu_launches": ((11 if fp8 else (7 if thr else 5))
+                             + (reblock_launches(N, prefix) + 2 if rbl else 0)) * args.steps,
             "clocks": clock_info,
             "context": {"pages_rtx_pro_6000_sparse_ms": 30.7 if cfg["N"] == 37_740 else None},
         }

@@ -80,6 +80,14 @@ _SIGS = {
     "bsa_attend_fp8": (ctypes.c_int, [_P, _F8, _vp, _vp, _vp, _vp, _vp, _vp]),
     "bsa_forward_fp8_workspace_bytes": (ctypes.c_size_t, [_P]),
     "bsa_forward_fp8": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "bsa_threshold_capacity": (ctypes.c_int32, [_P]),
+    "bsa_select_threshold": (ctypes.c_int, [_P, ctypes.c_float, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_attend_lists_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "bsa_attend_lists": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, ctypes.c_int32, _vp, _vp, _vp,
+                                        _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "bsa_forward_threshold_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "bsa_forward_threshold": (ctypes.c_int, [_P, ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp,
+                                             ctypes.c_size_t, _vp]),
 }
 
 
@@ -276,6 +284,40 @@ def bsa_forward_fp8(p, Q, K, V, O, lse, workspace, stream=None):
                                  _stream(stream)), "bsa_forward_fp8")
 
 
+def bsa_threshold_capacity(p: bsa_params) -> int:
+    return lib().bsa_threshold_capacity(ctypes.byref(p))
+
+
+def bsa_select_threshold(p, tau, qpool, kpool, idx, cnt, stream=None):
+    _check(lib().bsa_select_threshold(ctypes.byref(p), float(tau), _ptr(qpool), _ptr(kpool),
+                                      _ptr(idx), _ptr(cnt), _stream(stream)),
+           "bsa_select_threshold")
+
+
+def bsa_attend_lists_workspace_bytes(p: bsa_params) -> int:
+    return lib().bsa_attend_lists_workspace_bytes(ctypes.byref(p))
+
+
+def bsa_attend_lists(p, Q, K, V, idx, cnt, ksum, vsum, bias, O, lse, workspace, stream=None):
+    """bsa_attend over variable-length lists; the row stride is idx's last dimension."""
+    _check(lib().bsa_attend_lists(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                                  int(idx.shape[-1]), _ptr(cnt), _ptr(ksum), _ptr(vsum),
+                                  _ptr(bias), _ptr(O), _ptr(lse), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+           "bsa_attend_lists")
+
+
+def bsa_forward_threshold_workspace_bytes(p: bsa_params) -> int:
+    return lib().bsa_forward_threshold_workspace_bytes(ctypes.byref(p))
+
+
+def bsa_forward_threshold(p, tau, Q, K, V, O, lse, workspace, stream=None):
+    _check(lib().bsa_forward_threshold(ctypes.byref(p), float(tau), _ptr(Q), _ptr(K), _ptr(V),
+                                       _ptr(O), _ptr(lse), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream)), "bsa_forward_threshold")
+
+
 def bsa_debug_expired_wait(dev_status, timeout_ns: int, stream=None):
     _check(lib().bsa_debug_expired_wait(_ptr(dev_status), int(timeout_ns), _stream(stream)),
            "bsa_debug_expired_wait")
@@ -361,6 +403,21 @@ def forward_fp8(Q, K, V, top_k, prefix=0, variant="anchor", return_lse=False, ws
     if ws is None:
         ws = torch.empty(bsa_forward_fp8_workspace_bytes(p), dtype=torch.uint8, device=Q.device)
     bsa_forward_fp8(p, Q, K, V, O, lse, ws, stream)
+    return (O, lse) if return_lse else O
+
+
+def forward_threshold(Q, K, V, tau, prefix=0, variant="anchor", return_lse=False, ws=None,
+                      stream=None):
+    """bsa_forward_threshold: block-sparse attention whose lists keep the key
+    blocks at least tau standard deviations above each row's mean score."""
+    B, H, N, D = Q.shape
+    p = params(B, H, N, 1, prefix, variant, D=D)
+    O = torch.empty_like(Q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=Q.device) if return_lse else None
+    if ws is None:
+        ws = torch.empty(bsa_forward_threshold_workspace_bytes(p), dtype=torch.uint8,
+                         device=Q.device)
+    bsa_forward_threshold(p, tau, Q, K, V, O, lse, ws, stream)
     return (O, lse) if return_lse else O
 
 

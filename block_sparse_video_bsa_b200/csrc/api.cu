@@ -2,6 +2,7 @@
 // tensor-map construction and the launches of the four stages.  No memory is
 // allocated here and no state is kept between calls except per-device
 // capability / attribute caches.
+#include <cmath>
 #include <mutex>
 
 #include "bsa.h"
@@ -226,6 +227,27 @@ int attend_impl(const Shape& s, const void* Q, const void* K, const void* V, con
       !make_map(&maps.vs, vsum, s.nb, bh))
     return BSA_ERR_UNSUPPORTED;
   return cuda_status(bsa::launch_attend(s, maps, idx, cnt, bias, O, lse, st));
+}
+
+int attend_lists_impl(const Shape& s, const void* Q, const void* K, const void* V,
+                      const int32_t* idx, int kcap, const int32_t* cnt, const void* ksum,
+                      const void* vsum, const float* bias, void* O, float* lse, void* scratch,
+                      cudaStream_t st) {
+  bsa::AttendMaps maps;
+  const uint64_t bh = static_cast<uint64_t>(s.B) * s.H;
+  if (!make_map(&maps.q, Q, s.N, bh) || !make_map(&maps.k, K, s.N, bh) ||
+      !make_map(&maps.v, V, s.N, bh) || !make_map(&maps.ks, ksum, s.nb, bh) ||
+      !make_map(&maps.vs, vsum, s.nb, bh))
+    return BSA_ERR_UNSUPPORTED;
+  return cuda_status(
+      bsa::launch_attend_lists(s, maps, idx, kcap, cnt, bias, O, lse, scratch, st));
+}
+
+// The shape of a threshold call: list rows hold up to nb blocks.
+Shape threshold_shape(const Shape& s) {
+  Shape t = s;
+  t.kcap = s.nb;
+  return t;
 }
 
 // Reblocking scratch carved from one buffer (each piece 256-byte aligned).
@@ -491,6 +513,82 @@ int bsa_forward_fp8(const bsa_params* p, const void* Q, const void* K, const voi
   if ((rc = select_impl(s, w.qpool, w.kpool, w.idx, w.cnt, st))) return rc;
   if ((rc = quantize_fp8_impl(s, Q, K, V, w.ksum, w.vsum, f, st))) return rc;
   return attend_fp8_impl(s, f, w.idx, w.bias, O, lse, st);
+}
+
+int32_t bsa_threshold_capacity(const bsa_params* p) {
+  Shape s;
+  return shape_of(p, &s) == BSA_OK ? s.nb : -1;
+}
+
+int bsa_select_threshold(const bsa_params* p, float tau, const float* qpool, const float* kpool,
+                         int32_t* idx, int32_t* cnt, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!std::isfinite(tau) || !qpool || !kpool || !idx || !cnt) return BSA_ERR_INVALID;
+  if (!aligned(qpool, 16) || !aligned(kpool, 16) || !aligned(idx, 4) || !aligned(cnt, 4))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return cuda_status(bsa::launch_select_threshold(s, tau, qpool, kpool, idx, cnt,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+size_t bsa_attend_lists_workspace_bytes(const bsa_params* p) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK) return 0;
+  return bsa::attend_lists_scratch_bytes(s);
+}
+
+int bsa_attend_lists(const bsa_params* p, const void* Q, const void* K, const void* V,
+                     const int32_t* idx, int32_t kcap, const int32_t* cnt, const void* ksum,
+                     const void* vsum, const float* bias, void* O, float* lse, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !K || !V || !idx || !cnt || !ksum || !vsum || !bias || !O || !workspace)
+    return BSA_ERR_INVALID;
+  // prefix rows list all nb blocks, so a row must have room for them
+  if (kcap < (s.pb > 0 ? s.nb : 1) || kcap > s.nb) return BSA_ERR_INVALID;
+  if (workspace_bytes < bsa::attend_lists_scratch_bytes(s)) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(ksum, 16) ||
+      !aligned(vsum, 16) || !aligned(O, 16) || !aligned(idx, 4) || !aligned(cnt, 4) ||
+      !aligned(bias, 4) || !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return attend_lists_impl(s, Q, K, V, idx, kcap, cnt, ksum, vsum, bias, O, lse, workspace,
+                           static_cast<cudaStream_t>(stream));
+}
+
+size_t bsa_forward_threshold_workspace_bytes(const bsa_params* p) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK) return 0;
+  return carve(threshold_shape(s), nullptr, nullptr) + bsa::attend_lists_scratch_bytes(s);
+}
+
+int bsa_forward_threshold(const bsa_params* p, float tau, const void* Q, const void* K,
+                          const void* V, void* O, float* lse, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!std::isfinite(tau) || !Q || !K || !V || !O || !workspace) return BSA_ERR_INVALID;
+  const Shape t = threshold_shape(s);
+  const size_t ws0 = carve(t, nullptr, nullptr);
+  if (workspace_bytes < ws0 + bsa::attend_lists_scratch_bytes(s)) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
+      !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  Workspace w;
+  carve(t, static_cast<uint8_t*>(workspace), &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = pool_impl(s, Q, w.qpool, w.anchor, st))) return rc;
+  if ((rc = summarize_impl(s, K, V, w.anchor, w.kpool, w.ksum, w.vsum, w.bias, st))) return rc;
+  if ((rc = cuda_status(bsa::launch_select_threshold(s, tau, w.qpool, w.kpool, w.idx, w.cnt, st))))
+    return rc;
+  return attend_lists_impl(s, Q, K, V, w.idx, s.nb, w.cnt, w.ksum, w.vsum, w.bias, O, lse,
+                           static_cast<uint8_t*>(workspace) + ws0, st);
 }
 
 int32_t bsa_num_blocks(const bsa_params* p) {

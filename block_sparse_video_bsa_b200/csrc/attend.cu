@@ -11,9 +11,12 @@
 //     (compressed branch),
 // through one online softmax, so both branches share the running max and sum.
 //
-// Each CTA runs TWO query blocks ("slots") of the same tile count side by
-// side, so the tensor core works on one slot while the other slot's softmax
-// runs.  384 threads in three warpgroups; the two softmax warpgroups raise
+// Each CTA runs TWO query blocks ("slots") side by side, so the tensor core
+// works on one slot while the other slot's softmax runs.  With a fixed count
+// (top-k lists) both slots have the same tile count.  With variable-length
+// lists (kVar: the count of each row from cnt) each slot runs its own count;
+// the producer and the MMA issuer skip a slot once its tiles are done, and a
+// schedule sorted by count (longest first) pairs rows of similar length.  384 threads in three warpgroups; the two softmax warpgroups raise
 // their register budget to 232 and the third lowers its own to 40
 // (128*40 + 256*232 = 384*168, the launch allocation):
 //   warps 0-3   softmax of slot 0, one thread per query row (TMEM lanes 0-127)
@@ -74,6 +77,8 @@ static_assert(kOffCtl + sizeof(Ctl) <= 227 * 1024, "shared memory budget");
 
 struct Args {
   const int32_t* idx;
+  const int32_t* cnt;     // list lengths [B*H, nb] (kVar)
+  const int32_t* sched;   // video work items, longest list first (kVar)
   const float* bias;
   __nv_bfloat16* O;
   float* lse;
@@ -88,13 +93,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 // Pair of work items of one CTA: items 2c and 2c+1 of one class (dense-prefix
-// query blocks first, then video query blocks, head-major), so both slots
-// have the same tile count.
+// query blocks first, then video query blocks, head-major; with a schedule,
+// the video items in its order).
 struct Pair {
   int bh[2], qi[2];
   bool act1;
 };
 
+template <bool kVar>
 __device__ __forceinline__ Pair pair_of(int cta, const Args& a) {
   Pair p;
   int base, count, per_head, q0;
@@ -110,8 +116,10 @@ __device__ __forceinline__ Pair pair_of(int cta, const Args& a) {
     q0 = a.pb;
   }
   p.act1 = base + 1 < count;
+  const bool video = cta >= a.prefix_ctas;
   for (int s = 0; s < 2; ++s) {
-    const int it = min(base + s, count - 1);
+    int it = min(base + s, count - 1);
+    if (kVar && video) it = min(max(__ldg(a.sched + it), 0), count - 1);
     p.bh[s] = it / per_head;
     p.qi[s] = q0 + (it - p.bh[s] * per_head);
   }
@@ -129,6 +137,15 @@ __device__ __forceinline__ bool listed(const int32_t* row, int lo, int hi, int j
   return false;
 }
 
+// Listed blocks of a video row with a variable-length list, clamped to the
+// row's storage (at least one, so the tile loops and the ragged check stay
+// inside the row).
+__device__ __forceinline__ int list_len(const Args& a, int bh, int qi) {
+  const int c = __ldg(a.cnt + static_cast<size_t>(bh) * a.nb + qi);
+  return max(1, min(c, min(a.kcap, a.nb)));
+}
+
+template <bool kVar>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ks,
@@ -150,13 +167,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (ctl->skip) return;
 
-  const Pair pr = pair_of(blockIdx.x, a);
+  const Pair pr = pair_of<kVar>(blockIdx.x, a);
   const bool video = pr.qi[0] >= a.pb;
-  const int n_exact = video ? a.pb + a.k_eff : a.nb;
-  const bool has_sum = video && (a.k_eff < a.nbv);
   const int u0 = a.pb / kBlock;
-  const int T = n_exact + (has_sum ? ((a.nb + kBlock - 1) / kBlock - u0) : 0);
+  const int sum_tiles = (a.nb + kBlock - 1) / kBlock - u0;
+  // Per slot: listed blocks, whether summaries follow, tiles in all.
+  int ne0 = video ? a.pb + a.k_eff : a.nb, ne1 = ne0;
+  if (kVar && video) {
+    ne0 = list_len(a, pr.bh[0], pr.qi[0]);
+    ne1 = list_len(a, pr.bh[1], pr.qi[1]);
+  }
+  const bool hs0 = video && (ne0 - a.pb < a.nbv), hs1 = video && (ne1 - a.pb < a.nbv);
+  const int T0 = ne0 + (hs0 ? sum_tiles : 0), T1 = ne1 + (hs1 ? sum_tiles : 0);
   const int nslots = pr.act1 ? 2 : 1;
+  const int steps = (nslots == 2) ? max(T0, T1) : T0;   // tile steps of the CTA
+  auto n_exact_of = [&](int s) { return s ? ne1 : ne0; };
+  auto tiles_of = [&](int s) { return s ? T1 : T0; };
+  auto has_sum_of = [&](int s) { return s ? hs1 : hs0; };
 
   if (tid == 0) {
     for (int i = 0; i < kRing; ++i) {
@@ -213,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const CUtensorMap* m;
         int row;
+        const int n_exact = n_exact_of(s);
         if (t < n_exact) {
           row = __ldg(a.idx + (static_cast<size_t>(pr.bh[s]) * a.nb + pr.qi[s]) * a.kcap + t) *
                 kBlock;
@@ -228,10 +256,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++seq;
       };
       for (int s = 0; s < nslots; ++s) emit(s, 0, false);
-      for (int t = 0; t < T && ok; ++t) {
+      for (int t = 0; t < steps && ok; ++t) {
         for (int s = 0; s < nslots; ++s) {
+          if (t >= tiles_of(s)) continue;
           emit(s, t, true);
-          if (t + 1 < T) emit(s, t + 1, false);
+          if (t + 1 < tiles_of(s)) emit(s, t + 1, false);
         }
       }
       // Drain: every issued load has landed before the CTA exits (immediate
@@ -287,26 +316,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&ctl->q_full[s], 0, wc)) ok = false;
       }
       for (int s = 0; s < nslots && ok; ++s) issue_s(s);
-      for (int t = 0; t < T && ok; ++t) {
+      for (int t = 0; t < steps && ok; ++t) {
         for (int s = 0; s < nslots && ok; ++s) {
+          if (t >= tiles_of(s)) continue;
           issue_pv(s, t);
           if (!ok) break;
-          if (t + 1 < T) issue_s(s);
+          if (t + 1 < tiles_of(s)) issue_s(s);
           else mma_commit(&ctl->o_final[s]);
         }
       }
       mma_commit(&ctl->fin);
       mbar_wait(&ctl->fin, 0, wc);
-    } else if (warp >= 10 && has_sum && warp - 10 < nslots) {
+    } else if (warp >= 10 && warp - 10 < nslots && has_sum_of(warp - 10)) {
     // ---------------------------------------------------------- bias stager
       // Warp 10 + s stages, for each summary tile v of slot s, the 128 biases
       // in log2 units with -inf where the column is a listed block, a prefix
       // block or past the last block (listed: binary search of the sorted
       // idx row), double buffered against the slot's softmax warps.
       const int s = warp - 10;
+      const int n_exact = n_exact_of(s);
       const int32_t* idx_row = a.idx + (static_cast<size_t>(pr.bh[s]) * a.nb + pr.qi[s]) * a.kcap;
       const float* bias_h = a.bias + static_cast<size_t>(pr.bh[s]) * a.nb;
-      for (int v = 0; v < T - n_exact; ++v) {
+      for (int v = 0; v < tiles_of(s) - n_exact; ++v) {
         if (v >= 2 && !warp_wait(&ctl->bias_empty[s][v & 1], ((v >> 1) - 1) & 1, wc)) break;
         float* dst = &ctl->bias_stage[s][v & 1][0];
 #pragma unroll 1
@@ -331,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_col = tmem + lane_base + kColS + s * 128;
     const uint32_t o_col = tmem + lane_base + kColO + s * 128;
     const int bh = pr.bh[s], qi = pr.qi[s];
+    const int n_exact = n_exact_of(s), T = tiles_of(s);
     const int32_t* idx_row = a.idx + (static_cast<size_t>(bh) * a.nb + qi) * a.kcap;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = active;
@@ -485,24 +517,30 @@ __global__ void expired_wait_kernel(int* dev_status, uint64_t timeout_ns) {
 
 }  // namespace
 
-cudaError_t launch_attend(const Shape& s, const AttendMaps& maps, const int32_t* idx,
-                          const int32_t* cnt, const float* bias, void* O, float* lse,
-                          cudaStream_t st) {
-  // Tile counts follow from (pb, k_eff, nb): bsa_select lists pb + k_eff
-  // blocks for every video query block and all nb for a prefix block.
-  (void)cnt;
+namespace {
+
+// Shared setup of both launches: the kernel's shared-memory attribute (once
+// per device and instantiation) and the arguments common to both.
+template <bool kVar>
+cudaError_t attend_attr() {
   constexpr size_t smem = kOffCtl + sizeof(Ctl);
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(attend_kernel<kVar>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  return cudaSuccess;
+}
+
+Args attend_args(const Shape& s, const int32_t* idx, const float* bias, void* O, float* lse) {
   Args a;
   a.idx = idx;
+  a.cnt = nullptr;
+  a.sched = nullptr;
   a.bias = bias;
   a.O = static_cast<__nv_bfloat16*>(O);
   a.lse = lse;
@@ -516,8 +554,142 @@ cudaError_t launch_attend(const Shape& s, const AttendMaps& maps, const int32_t*
   a.BH = s.B * s.H;
   a.prefix_ctas = (a.BH * s.pb + 1) / 2;
   a.scale_log2 = kLog2e * 0.088388347648318440550f;
+  return a;
+}
+
+// ---------------------------------------------------------------- schedule
+// Video work items (bh * nbv + qi - pb) ordered by list length, longest
+// first, so that the two slots of a CTA hold rows of similar length and the
+// longest rows start first.  A counting sort: per-CTA shared-memory
+// histograms summed into `bins`, then every CTA scans `bins` from the
+// longest length down, reserves a range per length with one global atomic
+// and scatters its items.  The order inside one length follows the atomics;
+// no row's result depends on the row it is paired with.
+constexpr int kSchedThreads = 512;
+constexpr int kSchedItems = 8192;        // items per CTA
+
+__device__ __forceinline__ int item_len(const int32_t* cnt, int it, int nbv, int nb, int pb,
+                                        int kcap) {
+  const int bh = it / nbv, qi = pb + (it - bh * nbv);
+  const int c = __ldg(cnt + static_cast<size_t>(bh) * nb + qi);
+  return max(1, min(c, min(kcap, nb)));
+}
+
+__global__ void __launch_bounds__(kSchedThreads)
+    length_hist_kernel(const int32_t* __restrict__ cnt, int items, int nbv, int nb, int pb,
+                       int kcap, int32_t* __restrict__ bins) {
+  extern __shared__ int h[];             // [nb + 1]
+  for (int b = threadIdx.x; b <= nb; b += kSchedThreads) h[b] = 0;
+  __syncthreads();
+  const int i0 = blockIdx.x * kSchedItems, i1 = min(items, i0 + kSchedItems);
+  for (int it = i0 + threadIdx.x; it < i1; it += kSchedThreads)
+    atomicAdd(&h[item_len(cnt, it, nbv, nb, pb, kcap)], 1);
+  __syncthreads();
+  for (int b = threadIdx.x; b <= nb; b += kSchedThreads)
+    if (h[b]) atomicAdd(&bins[b], h[b]);
+}
+
+__global__ void __launch_bounds__(kSchedThreads)
+    schedule_kernel(const int32_t* __restrict__ cnt, int items, int nbv, int nb, int pb, int kcap,
+                    const int32_t* __restrict__ bins, int32_t* __restrict__ fill,
+                    int32_t* __restrict__ sched) {
+  extern __shared__ int sm_sched[];
+  int* start = sm_sched;                 // [nb + 1] items with a longer list
+  int* cur = sm_sched + (nb + 1);        // [nb + 1] local counts, then cursors
+  __shared__ int part[kSchedThreads];
+  const int tid = threadIdx.x, nbins = nb + 1;
+  // start[b] = sum of bins[b'] over b' > b: thread t scans a contiguous run
+  // of the reversed bins, then the run totals are scanned across the block.
+  const int per = (nbins + kSchedThreads - 1) / kSchedThreads;
+  const int r0 = min(nbins, tid * per), r1 = min(nbins, r0 + per);
+  int run = 0;
+  for (int r = r0; r < r1; ++r) run += __ldg(bins + (nb - r));
+  part[tid] = run;
+  for (int b = tid; b < nbins; b += kSchedThreads) cur[b] = 0;
+  __syncthreads();
+  for (int off = 1; off < kSchedThreads; off <<= 1) {      // inclusive scan of part
+    const int v = tid >= off ? part[tid - off] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  int acc = part[tid] - run;                                // exclusive prefix of the run
+  for (int r = r0; r < r1; ++r) {
+    start[nb - r] = acc;
+    acc += __ldg(bins + (nb - r));
+  }
+  const int i0 = blockIdx.x * kSchedItems, i1 = min(items, i0 + kSchedItems);
+  for (int it = i0 + tid; it < i1; it += kSchedThreads)
+    atomicAdd(&cur[item_len(cnt, it, nbv, nb, pb, kcap)], 1);
+  __syncthreads();
+  for (int b = tid; b < nbins; b += kSchedThreads)
+    if (cur[b]) cur[b] = start[b] + atomicAdd(&fill[b], cur[b]);
+  __syncthreads();
+  for (int it = i0 + tid; it < i1; it += kSchedThreads) {
+    const int pos = atomicAdd(&cur[item_len(cnt, it, nbv, nb, pb, kcap)], 1);
+    if (pos >= 0 && pos < items) sched[pos] = it;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attend(const Shape& s, const AttendMaps& maps, const int32_t* idx,
+                          const int32_t* cnt, const float* bias, void* O, float* lse,
+                          cudaStream_t st) {
+  // Tile counts follow from (pb, k_eff, nb): bsa_select lists pb + k_eff
+  // blocks for every video query block and all nb for a prefix block.
+  (void)cnt;
+  cudaError_t e = attend_attr<false>();
+  if (e != cudaSuccess) return e;
+  const Args a = attend_args(s, idx, bias, O, lse);
   const int grid = a.prefix_ctas + (a.BH * s.nbv + 1) / 2;
-  attend_kernel<<<grid, kThreads, smem, st>>>(maps.q, maps.k, maps.v, maps.ks, maps.vs, a);
+  attend_kernel<false><<<grid, kThreads, kOffCtl + sizeof(Ctl), st>>>(maps.q, maps.k, maps.v,
+                                                                      maps.ks, maps.vs, a);
+  return cudaGetLastError();
+}
+
+size_t attend_lists_scratch_bytes(const Shape& s) {
+  const size_t bins = (static_cast<size_t>(s.nb) + 1) * 4;
+  return 2 * ((bins + 255) & ~static_cast<size_t>(255)) +
+         static_cast<size_t>(s.B) * s.H * s.nbv * 4;
+}
+
+cudaError_t launch_attend_lists(const Shape& s, const AttendMaps& maps, const int32_t* idx,
+                                int kcap, const int32_t* cnt, const float* bias, void* O,
+                                float* lse, void* scratch, cudaStream_t st) {
+  cudaError_t e = attend_attr<true>();
+  if (e != cudaSuccess) return e;
+  const size_t smem_sched = 2 * (static_cast<size_t>(s.nb) + 1) * sizeof(int);
+  static bool sched_attr[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !sched_attr[dev]) {
+    const int max_dyn = 2 * (16384 + 1) * static_cast<int>(sizeof(int));
+    if ((e = cudaFuncSetAttribute(length_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  max_dyn)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  max_dyn)) != cudaSuccess)
+      return e;
+    sched_attr[dev] = true;
+  }
+  const size_t bins_bytes = ((static_cast<size_t>(s.nb) + 1) * 4 + 255) & ~static_cast<size_t>(255);
+  int32_t* bins = static_cast<int32_t*>(scratch);
+  int32_t* fill = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + bins_bytes);
+  int32_t* sched = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + 2 * bins_bytes);
+  const int items = s.B * s.H * s.nbv;
+  if ((e = cudaMemsetAsync(scratch, 0, 2 * bins_bytes, st)) != cudaSuccess) return e;
+  const int sched_grid = (items + kSchedItems - 1) / kSchedItems;
+  length_hist_kernel<<<sched_grid, kSchedThreads, (s.nb + 1) * sizeof(int), st>>>(
+      cnt, items, s.nbv, s.nb, s.pb, kcap, bins);
+  schedule_kernel<<<sched_grid, kSchedThreads, smem_sched, st>>>(cnt, items, s.nbv, s.nb, s.pb,
+                                                                 kcap, bins, fill, sched);
+  Args a = attend_args(s, idx, bias, O, lse);
+  a.cnt = cnt;
+  a.sched = sched;
+  a.kcap = kcap;
+  const int grid = a.prefix_ctas + (a.BH * s.nbv + 1) / 2;
+  attend_kernel<true><<<grid, kThreads, kOffCtl + sizeof(Ctl), st>>>(maps.q, maps.k, maps.v,
+                                                                     maps.ks, maps.vs, a);
   return cudaGetLastError();
 }
 

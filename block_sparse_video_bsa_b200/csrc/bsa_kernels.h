@@ -26,6 +26,10 @@ cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const
                              float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st);
 cudaError_t launch_select(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
                           int32_t* cnt, cudaStream_t st);
+// Threshold selection: idx rows of length nb (kcap ignored), cnt per row.
+cudaError_t launch_select_threshold(const Shape& s, float tau, const float* qpool,
+                                    const float* kpool, int32_t* idx, int32_t* cnt,
+                                    cudaStream_t st);
 
 struct AttendMaps {
   CUtensorMap q, k, v, ks, vs;   // bf16, box {64, 128, 1}, 128B swizzle
@@ -33,6 +37,12 @@ struct AttendMaps {
 cudaError_t launch_attend(const Shape& s, const AttendMaps& maps, const int32_t* idx,
                           const int32_t* cnt, const float* bias, void* O, float* lse,
                           cudaStream_t st);
+// Variable-length lists (row stride kcap, length cnt per row); `scratch`
+// holds the schedule (attend_lists_scratch_bytes).
+size_t attend_lists_scratch_bytes(const Shape& s);
+cudaError_t launch_attend_lists(const Shape& s, const AttendMaps& maps, const int32_t* idx,
+                                int kcap, const int32_t* cnt, const float* bias, void* O,
+                                float* lse, void* scratch, cudaStream_t st);
 // FP8 (e4m3) operands (layouts as bsa_fp8_operands in include/bsa.h).
 struct Fp8Operands {
   void* q8;

@@ -16,6 +16,13 @@
 //     lowest-index blocks equal to it -- exactly "score descending, ties to
 //     the lower index".
 // Dense-prefix query blocks (i < pb) list every block.
+//
+// Threshold mode (content-adaptive count; "H3 Sparse Attention", WAS node
+// page, "The inputs that matter": the kept share of key blocks is set by a
+// threshold tau): phase 2 keeps, per query block, the video key blocks whose
+// score is at least tau population standard deviations above the row's mean
+// (all of them when the row's scores are all equal, the top-scoring one when
+// none qualifies), so list lengths vary from row to row.
 #include "bsa_device.cuh"
 #include "bsa_kernels.h"
 
@@ -103,12 +110,67 @@ __device__ __forceinline__ void topk_row_smem(const float* srow, int nbv, int k_
   }
 }
 
-template <int kPerLane>   // 0 = keys stay in shared memory
+// Threshold selection of one row of nbv scores (in shared memory) by one
+// warp.  The sums are xor-butterfly reductions, so every lane holds the same
+// bits of the mean and deviation and takes the same decisions.  Writes the
+// kept blocks in ascending order at row[pb...] and returns how many.
+__device__ __forceinline__ int threshold_row(const float* srow, int nbv, float tau, int pb,
+                                             int32_t* row, int lane) {
+  float sum = 0.f, mx = -INFINITY, mn = INFINITY;
+  for (int j = lane; j < nbv; j += 32) {
+    const float x = srow[j];
+    sum += x;
+    mx = fmaxf(mx, x);
+    mn = fminf(mn, x);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  const float mean = sum / static_cast<float>(nbv);
+  float ss = 0.f;
+  for (int j = lane; j < nbv; j += 32) {
+    const float dev = srow[j] - mean;
+    ss = fmaf(dev, dev, ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float margin = tau * sqrtf(ss / static_cast<float>(nbv));
+  const bool all = (mx == mn);           // no contrast: every block
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int out = 0;
+  for (int base = 0; base < nbv; base += 32) {
+    const int j = base + lane;
+    const bool sel = j < nbv && (all || srow[j] - mean >= margin);
+    const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+    if (sel) row[pb + out + __popc(selm & lt_mask)] = pb + j;
+    out += __popc(selm);
+  }
+  if (out == 0) {
+    // floor: the first block whose score equals the row maximum
+    int first = nbv;
+    for (int base = 0; base < nbv && first == nbv; base += 32) {
+      const int j = base + lane;
+      const uint32_t m = __ballot_sync(0xffffffffu, j < nbv && srow[j] == mx);
+      if (m) first = base + __ffs(m) - 1;
+    }
+    if (lane == 0) row[pb] = pb + min(first, nbv - 1);
+    out = 1;
+  }
+  return out;
+}
+
+// kPerLane: keys per lane of the top-k search (0 = keys stay in shared
+// memory); kThresh: threshold mode (tau used, k_eff unused, kcap = nb).
+template <int kPerLane, bool kThresh>
 __global__ void __launch_bounds__(kThreads) select_kernel(const float* __restrict__ qpool,
                                                           const float* __restrict__ kpool,
                                                           int32_t* __restrict__ idx,
                                                           int32_t* __restrict__ cnt, int nb, int pb,
-                                                          int k_eff, int kcap, int R, float scale) {
+                                                          int k_eff, int kcap, int R, float scale,
+                                                          float tau) {
   extern __shared__ float smem[];
   const int nbv = nb - pb;
   float* qp = smem;                          // [R][kPad]
@@ -172,32 +234,37 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float* __restric
       if (lane == 0) cnt[bh * nb + i] = nb;
       continue;
     }
-    if (kPerLane > 0)
-      topk_row<(kPerLane > 0 ? kPerLane : 1)>(sc + r * nbv, nbv, k_eff, pb, row, lane);
+    int kept = k_eff;
+    if constexpr (kThresh)
+      kept = threshold_row(sc + r * nbv, nbv, tau, pb, row, lane);
+    else if constexpr (kPerLane > 0)
+      topk_row<kPerLane>(sc + r * nbv, nbv, k_eff, pb, row, lane);
     else
       topk_row_smem(sc + r * nbv, nbv, k_eff, pb, row, lane);
     for (int p = lane; p < pb; p += 32) row[p] = p;
-    for (int p = pb + k_eff + lane; p < kcap; p += 32) row[p] = -1;
-    if (lane == 0) cnt[bh * nb + i] = pb + k_eff;
+    for (int p = pb + kept + lane; p < kcap; p += 32) row[p] = -1;
+    if (lane == 0) cnt[bh * nb + i] = pb + kept;
   }
 }
 
-template <int kPerLane>
+template <int kPerLane, bool kThresh = false>
 cudaError_t launch_select_t(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
-                            int32_t* cnt, int R, size_t smem, cudaStream_t st) {
+                            int32_t* cnt, int R, size_t smem, cudaStream_t st, float tau = 0.f) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel<kPerLane>,
+    cudaError_t e = cudaFuncSetAttribute(select_kernel<kPerLane, kThresh>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   const dim3 grid((s.nb + R - 1) / R, s.B * s.H);
   const float scale = 0.088388347648318440550f;
-  select_kernel<kPerLane><<<grid, kThreads, smem, st>>>(qpool, kpool, idx, cnt, s.nb, s.pb,
-                                                        s.k_eff, s.kcap, R, scale);
+  const int kcap = kThresh ? s.nb : s.kcap;
+  select_kernel<kPerLane, kThresh><<<grid, kThreads, smem, st>>>(qpool, kpool, idx, cnt, s.nb,
+                                                                 s.pb, s.k_eff, kcap, R, scale,
+                                                                 tau);
   return cudaGetLastError();
 }
 
@@ -212,11 +279,22 @@ static int select_rows(int nbv) {
   return R;
 }
 
+static size_t select_smem(int R, int nbv) {
+  return (static_cast<size_t>(R) * kPad + kChunk * kPad + static_cast<size_t>(R) * nbv) *
+         sizeof(float);
+}
+
+cudaError_t launch_select_threshold(const Shape& s, float tau, const float* qpool,
+                                    const float* kpool, int32_t* idx, int32_t* cnt,
+                                    cudaStream_t st) {
+  const int R = select_rows(s.nbv);
+  return launch_select_t<0, true>(s, qpool, kpool, idx, cnt, R, select_smem(R, s.nbv), st, tau);
+}
+
 cudaError_t launch_select(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
                           int32_t* cnt, cudaStream_t st) {
   const int R = select_rows(s.nbv);
-  const size_t smem = (static_cast<size_t>(R) * kPad + kChunk * kPad + static_cast<size_t>(R) * s.nbv) *
-                      sizeof(float);
+  const size_t smem = select_smem(R, s.nbv);
   // keys per lane: the smallest instantiation that holds the row
   if (s.nbv <= 32 * 8) return launch_select_t<8>(s, qpool, kpool, idx, cnt, R, smem, st);
   if (s.nbv <= 32 * 12) return launch_select_t<12>(s, qpool, kpool, idx, cnt, R, smem, st);

@@ -305,6 +305,57 @@ int bsa_forward_fp8(const bsa_params* p, const void* Q, const void* K, const voi
                     void* O, float* lse, void* workspace, size_t workspace_bytes,
                     void* stream);
 
+/* ---- option: threshold selection (content-adaptive count) ---------------
+ * "H3 Sparse Attention" (comfy.icu, WAS node page), "The inputs that
+ * matter": the content-adaptive method takes a threshold tau instead of a
+ * block count, and keeps about 16 %, 7 % and 3 % of the key blocks at
+ * tau = 1.0, 1.5 and 2.0 -- the standard normal's upper tail at tau, so the
+ * threshold is read as a z-score of the pooled block scores.  Lists then
+ * vary in length from row to row; p->top_k is not used by these calls
+ * (any value >= 1). */
+
+/* Row length of the idx array written by bsa_select_threshold: nb. */
+int32_t bsa_threshold_capacity(const bsa_params* p);
+
+/* Steps 4-5 with threshold selection.  For video query block i >= pb, with
+ * S_ij as in bsa_select over the video key blocks j in [pb, nb), mu_i their
+ * mean and sigma_i their population standard deviation (fp32): keep every j
+ * with S_ij - mu_i >= tau * sigma_i; every j when the row's scores are all
+ * equal; the top-scoring j (lowest index on ties) when none qualifies.
+ *   idx[b,h,i,:] = 0..pb-1, then the kept j ascending, then -1 padding
+ *   (int32 [B,H,nb,nb]),  cnt[b,h,i] = pb + number kept  (int32 [B,H,nb]).
+ * Prefix query blocks list every block, as in bsa_select.  tau must be
+ * finite (else BSA_ERR_INVALID).  Deterministic. */
+int bsa_select_threshold(const bsa_params* p, float tau, const float* qpool,
+                         const float* kpool, int32_t* idx, int32_t* cnt, void* stream);
+
+/* Scratch of bsa_attend_lists (the work schedule): bytes, or 0 if p is
+ * invalid. */
+size_t bsa_attend_lists_workspace_bytes(const bsa_params* p);
+
+/* Step 6 over variable-length lists: as bsa_attend, but row i of idx has
+ * stride kcap and holds cnt[b,h,i] listed blocks (ascending, the pb prefix
+ * blocks first; prefix query blocks list all nb).  Counts are clamped to
+ * [1, kcap].  Requires kcap <= nb, and kcap == nb when prefix > 0
+ * (BSA_ERR_INVALID otherwise).  `workspace` (device, 256-byte aligned, at
+ * least bsa_attend_lists_workspace_bytes(p) bytes) holds the schedule that
+ * pairs rows of similar length; its contents need not be initialised.
+ * Deterministic: no row's result depends on the rows it is scheduled with. */
+int bsa_attend_lists(const bsa_params* p, const void* Q, const void* K, const void* V,
+                     const int32_t* idx, int32_t kcap, const int32_t* cnt,
+                     const void* ksum, const void* vsum, const float* bias, void* O,
+                     float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace of bsa_forward_threshold. */
+size_t bsa_forward_threshold_workspace_bytes(const bsa_params* p);
+
+/* bsa_pool, bsa_summarize, bsa_select_threshold, bsa_attend_lists in order on
+ * `stream`, intermediates in the caller's workspace (256-byte aligned, at
+ * least bsa_forward_threshold_workspace_bytes(p) bytes). */
+int bsa_forward_threshold(const bsa_params* p, float tau, const void* Q, const void* K,
+                          const void* V, void* O, float* lse, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
 /* Human-readable name of a bsa_status value (static string). */
 const char* bsa_status_string(int status);
 

@@ -97,11 +97,8 @@ def check_output(O_gpu, O_ref, N, exclude_blocks=()):
     return max_abs, rel_l2
 
 
-def check_head(buf, Q, K, V, b, h, top_k, prefix, variant, check_lse=True):
-    """Full per-stage parity of one (b, h) slice; returns (max_abs, rel_l2, swaps)."""
-    N = Q.shape[2]
-    ref = orc.forward_head(host(Q[b, h]), host(K[b, h]), host(V[b, h]), top_k, prefix, variant)
-    pb = prefix // 128
+def check_stages(buf, ref, b, h, pb):
+    """Pools, anchor, summaries and bias of one (b, h) slice vs the oracle."""
     np.testing.assert_allclose(host(buf["qpool"][b, h]), ref["qpool"], rtol=POOL_RTOL, atol=POOL_ATOL)
     np.testing.assert_allclose(host(buf["kpool"][b, h]), ref["kpool"], rtol=POOL_RTOL, atol=POOL_ATOL)
     np.testing.assert_allclose(host(buf["anchor"][b, h]), ref["anchor"], rtol=POOL_RTOL,
@@ -114,18 +111,121 @@ def check_head(buf, Q, K, V, b, h, top_k, prefix, variant, check_lse=True):
     bias_tol = BF16_U * (kabs @ np.abs(ref["anchor"])) / np.sqrt(d) + FP32_SLACK
     bias_err = np.abs(host(buf["bias"][b, h])[v] - ref["bias"][v])
     assert (bias_err <= bias_tol).all(), f"bias err {bias_err.max()} > {bias_tol.min()}"
+
+
+def check_lse_bound(lse_gpu, Qh, ref, lse_ref, pb, variant, N, exclude_blocks=()):
+    """lse within the bound the bf16 summary keys allow (oracle values only)."""
+    keep = np.ones(N, dtype=bool)
+    if exclude_blocks:
+        keep[rows_of_blocks(N, exclude_blocks)] = False
+    d = ref["ksum"].shape[1]
+    kabs = np.abs(ref["ksum"][pb:])
+    # anchor variant: the shift is (q - qbar) . delta; mean variant: q . delta
+    centre = ref["anchor"][None, :] if variant == "anchor" else 0.0
+    qd = np.abs(Qh - centre)
+    lse_tol = BF16_U * (qd @ kabs.T).max(axis=1) / np.sqrt(d) + FP32_SLACK \
+        if kabs.size else np.full(N, FP32_SLACK)
+    lse_err = np.abs(lse_gpu - lse_ref)
+    assert (lse_err[keep] <= lse_tol[keep]).all(), \
+        f"lse err {lse_err[keep].max()} (bound {lse_tol[keep].min()})"
+
+
+def check_head(buf, Q, K, V, b, h, top_k, prefix, variant, check_lse=True):
+    """Full per-stage parity of one (b, h) slice; returns (max_abs, rel_l2, swaps)."""
+    N = Q.shape[2]
+    ref = orc.forward_head(host(Q[b, h]), host(K[b, h]), host(V[b, h]), top_k, prefix, variant)
+    pb = prefix // 128
+    check_stages(buf, ref, b, h, pb)
     swaps = check_selection(host(buf["idx"][b, h]), host(buf["cnt"][b, h]), ref, pb, top_k)
     m, r = check_output(host(buf["O"][b, h]), ref["O"], N, swaps)
     if check_lse and buf.get("lse") is not None:
-        keep = np.ones(N, dtype=bool)
-        if swaps:
-            keep[rows_of_blocks(N, swaps)] = False
-        # anchor variant: the shift is (q - qbar) . delta; mean variant: q . delta
-        centre = ref["anchor"][None, :] if variant == "anchor" else 0.0
-        qd = np.abs(host(Q[b, h]) - centre)
-        lse_tol = BF16_U * (qd @ kabs.T).max(axis=1) / np.sqrt(d) + FP32_SLACK \
-            if kabs.size else np.full(N, FP32_SLACK)
-        lse_err = np.abs(host(buf["lse"][b, h]) - ref["lse"])
-        assert (lse_err[keep] <= lse_tol[keep]).all(), \
-            f"lse err {lse_err[keep].max()} (bound {lse_tol[keep].min()})"
+        check_lse_bound(host(buf["lse"][b, h]), host(Q[b, h]), ref, ref["lse"], pb, variant, N,
+                        swaps)
     return m, r, swaps
+
+
+# ------------------------------------------------------------ threshold lists
+
+# Band around a row's threshold (logit scale) inside which the GPU's fp32
+# statistic may decide a block either way: the fp32 scores are within ~1e-5 of
+# the fp64 ones (the top-k tie gap), and the mean and deviation add errors of
+# the same order times tau.
+THRESH_BAND = 1e-4
+
+
+def check_threshold_selection(idx_rows, cnt_row, S, tau, pb):
+    """GPU lists of one head vs the threshold oracle.  Returns the GPU's lists
+    (each checked for validity) and the rows where they differ from the
+    oracle's, which is allowed only for blocks within THRESH_BAND of the row's
+    threshold, or, where the oracle fell back to the top block, for a GPU top
+    block within the top-k tie gap of the row maximum."""
+    from oracle import bsa_oracle_threshold as th
+    nb = S.shape[0]
+    want_lists = th.select_blocks_threshold(S, tau, pb)
+    cand = np.arange(pb, nb)
+    got_lists, differ = [], set()
+    for i in range(nb):
+        c = int(cnt_row[i])
+        assert 1 <= c <= nb, (i, c)
+        got = [int(v) for v in idx_rows[i, :c]]
+        assert all(int(v) == -1 for v in idx_rows[i, c:]), f"padding of row {i}"
+        got_lists.append(np.array(got, dtype=np.int64))
+        want = [int(v) for v in want_lists[i]]
+        if got == want:
+            continue
+        assert i >= pb, f"prefix row {i} differs"
+        assert got[:pb] == list(range(pb))
+        assert got == sorted(set(got)) and all(pb <= j < nb for j in got[pb:]), i
+        row = S[i, cand]
+        mu, margin = th.row_threshold(row, tau)
+        floor = not np.any(row - mu >= margin) and row.max() != row.min()
+        if floor and len(got) == pb + 1 and S[i, got[-1]] >= row.max() - TIE_GAP:
+            differ.add(i)
+            continue
+        for j in set(got) ^ set(want):
+            assert abs(S[i, j] - mu - margin) <= THRESH_BAND, (i, j, S[i, j] - mu - margin)
+        differ.add(i)
+    return got_lists, differ
+
+
+def run_stages_threshold(Q, K, V, tau, prefix, variant, with_lse=True):
+    """The threshold path stage by stage through its C entry points."""
+    B, H, N, _ = Q.shape
+    p = bsa.params(B, H, N, 1, prefix, variant)
+    buf = bsa.stage_buffers(B, H, N, 1, prefix, variant, device=Q.device)
+    nb = bsa.bsa_num_blocks(p)
+    buf["idx"] = torch.empty(B, H, nb, bsa.bsa_threshold_capacity(p), dtype=torch.int32,
+                             device=Q.device)
+    bsa.bsa_pool(p, Q, buf["qpool"], buf["anchor"])
+    bsa.bsa_summarize(p, K, V, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"], buf["bias"])
+    bsa.bsa_select_threshold(p, tau, buf["qpool"], buf["kpool"], buf["idx"], buf["cnt"])
+    O = torch.empty_like(Q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=Q.device) if with_lse else None
+    ws = torch.empty(bsa.bsa_attend_lists_workspace_bytes(p), dtype=torch.uint8, device=Q.device)
+    bsa.bsa_attend_lists(p, Q, K, V, buf["idx"], buf["cnt"], buf["ksum"], buf["vsum"],
+                         buf["bias"], O, lse, ws)
+    torch.cuda.synchronize()
+    buf["O"] = O
+    buf["lse"] = lse
+    return buf
+
+
+def check_head_threshold(buf, Q, K, V, b, h, tau, prefix, variant, check_lse=True):
+    """Per-stage parity of one (b, h) slice of the threshold path: stages and
+    lists against the oracle, then O and lse against the oracle's attention
+    over the GPU's (validated) lists.  Returns (max_abs, rel_l2, rows that
+    differ, kept video blocks per row)."""
+    from oracle import bsa_oracle_threshold as th
+    N = Q.shape[2]
+    Qh, Kh, Vh = host(Q[b, h]), host(K[b, h]), host(V[b, h])
+    ref = th.forward_head_threshold(Qh, Kh, Vh, tau, prefix, variant, query_blocks=set())
+    pb = prefix // 128
+    check_stages(buf, ref, b, h, pb)
+    lists, differ = check_threshold_selection(host(buf["idx"][b, h]), host(buf["cnt"][b, h]),
+                                              ref["scores"], tau, pb)
+    O_ref, lse_ref = orc.attend(Qh, Kh, Vh, lists, ref["ksum"], ref["vsum"], ref["bias"], pb)
+    m, r = check_output(host(buf["O"][b, h]), O_ref, N)
+    if check_lse and buf.get("lse") is not None:
+        check_lse_bound(host(buf["lse"][b, h]), Qh, ref, lse_ref, pb, variant, N)
+    kept = np.array([len(l) - pb for l in lists[pb:]])
+    return m, r, differ, kept

@@ -172,3 +172,46 @@ def _reblock_scratch(B, H, N, prefix):
 def test_reblock_scratch_follows_the_tree_shape(B, H, N, prefix):
     p = bsa.params(B, H, N, 1, prefix)
     assert bsa.bsa_reblock_workspace_bytes(p) == _reblock_scratch(B, H, N, prefix)
+
+
+def test_threshold_sizes():
+    # lists of up to nb blocks; the schedule holds one int per video query
+    # block plus two length histograms
+    p = _p()
+    bh, nb = 56, 295
+    assert bsa.bsa_threshold_capacity(p) == nb
+    assert bsa.bsa_threshold_capacity(_p(top_k=0)) == -1
+    r256 = lambda x: (x + 255) // 256 * 256
+    assert bsa.bsa_attend_lists_workspace_bytes(p) == 2 * r256((nb + 1) * 4) + bh * nb * 4
+    pp = _p(N=103_996, prefix=512)
+    assert bsa.bsa_attend_lists_workspace_bytes(pp) == 2 * r256((813 + 1) * 4) + bh * 809 * 4
+    fw = bsa.bsa_forward_threshold_workspace_bytes(p)
+    fixed = bsa.bsa_workspace_bytes(p)             # idx rows of 64 there, of 295 here
+    assert fw - bsa.bsa_attend_lists_workspace_bytes(p) - fixed == \
+        r256(bh * nb * nb * 4) - r256(bh * nb * 64 * 4)
+
+
+def test_threshold_arguments_rejected_before_launch():
+    L = bsa.lib()
+    p = _p()
+    P = ctypes.byref(p)
+    a = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    big = 1 << 40
+    for tau in (float("nan"), float("inf"), float("-inf")):
+        assert L.bsa_select_threshold(P, tau, a, a, a, a, None) == bsa.BSA_ERR_INVALID
+        assert L.bsa_forward_threshold(P, tau, a, a, a, a, None, a, big, None) == \
+            bsa.BSA_ERR_INVALID
+    assert L.bsa_select_threshold(P, 1.0, a, a, None, a, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_select_threshold(P, 1.0, odd, a, a, a, None) == bsa.BSA_ERR_ALIGN
+    args = lambda kcap, ws=big, o=a, w=a: (P, a, a, a, a, kcap, a, a, a, a, o, None, w, ws, None)
+    assert L.bsa_attend_lists(*args(0)) == bsa.BSA_ERR_INVALID          # empty rows
+    assert L.bsa_attend_lists(*args(296)) == bsa.BSA_ERR_INVALID        # wider than nb
+    assert L.bsa_attend_lists(*args(295, ws=16)) == bsa.BSA_ERR_INVALID  # schedule too small
+    assert L.bsa_attend_lists(*args(295, o=odd)) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_attend_lists(*args(295, w=odd)) == bsa.BSA_ERR_ALIGN
+    # with a dense prefix the rows must hold all nb blocks
+    pp = _p(N=103_996, prefix=512)
+    assert L.bsa_attend_lists(ctypes.byref(pp), a, a, a, a, 812, a, a, a, a, a, None, a, big,
+                              None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_forward_threshold(P, 1.0, a, a, a, a, None, a, 16, None) == bsa.BSA_ERR_INVALID
