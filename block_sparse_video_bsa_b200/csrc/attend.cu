@@ -16,8 +16,9 @@
 // (top-k lists) both slots have the same tile count.  With variable-length
 // lists (kVar: the count of each row from cnt) each slot runs its own count;
 // the producer and the MMA issuer skip a slot once its tiles are done, and a
-// schedule sorted by count (longest first) pairs rows of similar length.  384 threads in three warpgroups; the two softmax warpgroups raise
-// their register budget to 232 and the third lowers its own to 40
+// schedule sorted by count (longest first) pairs rows of similar length.
+// 384 threads in three warpgroups; the two softmax warpgroups raise their
+// register budget to 232 and the third lowers its own to 40
 // (128*40 + 256*232 = 384*168, the launch allocation):
 //   warps 0-3   softmax of slot 0, one thread per query row (TMEM lanes 0-127)
 //   warps 4-7   softmax of slot 1
