@@ -87,3 +87,19 @@ def test_reference_arm_prints_its_line():
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["metric"] == bench.METRIC
+
+
+def test_threshold_options():
+    # --tau runs the bf16 path without reblocking; the reference arm times the
+    # threshold oracle on the same workload and names the selection.
+    for bad in (["--tau", "1.0", "--reblock"], ["--tau", "1.0", "--precision", "fp8"]):
+        out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *bad],
+                             capture_output=True, text=True, timeout=120, cwd=ROOT)
+        assert out.returncode != 0 and "--tau" in out.stderr
+    out = subprocess.run(
+        [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+         "tiny_iid", "--tau", "1.0", "--steps", "1", "--warmup", "0"],
+        capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    line = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
+    assert line["config"]["selection"] == "threshold tau=1.0" and line["value"] > 0
