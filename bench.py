@@ -306,6 +306,13 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+def data_label(cfg):
+    """What the timed inputs are: the seeded generator kind and the workload shape."""
+    kind = {"block_offset": "per-block-offset", "iid": "iid N(0,1)"}.get(cfg["kind"], cfg["kind"])
+    return (f"synthetic (seeded {kind} bf16 Q/K/V, workload {cfg['name']}: B={cfg['B']}, "
+            f"H={cfg['H']}, N={cfg['N']})")
+
+
 def config_block(cfg, **extra):
     d = {"workload": cfg["name"], "B": cfg["B"], "H": cfg["H"], "N": cfg["N"], "d": 128,
          "top_k": cfg["top_k"], "prefix": cfg["prefix"], "summary": cfg["variant"],
@@ -544,7 +551,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3" if fp8 else "bf16",
-            "data": "synthetic (seeded per-block-offset bf16 Q/K/V of the H3 768p-5s shape)",
+            "data": data_label(cfg),
             "config": config_block(cfg, parallelism=f"{world} independent calls (one per GPU)",
                                    **({"layout": "adaptive reblocking (q_reuse_k)"} if rbl
                                       else {}),

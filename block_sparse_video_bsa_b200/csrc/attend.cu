@@ -525,16 +525,11 @@ namespace {
 template <bool kVar>
 cudaError_t attend_attr() {
   constexpr size_t smem = kOffCtl + sizeof(Ctl);
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attend_kernel<kVar>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
-  return cudaSuccess;
+  static std::atomic<bool> attr_set[64];
+  return once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(attend_kernel<kVar>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem);
+  });
 }
 
 Args attend_args(const Shape& s, const int32_t* idx, const float* bias, void* O, float* lse) {
@@ -661,18 +656,16 @@ cudaError_t launch_attend_lists(const Shape& s, const AttendMaps& maps, const in
   cudaError_t e = attend_attr<true>();
   if (e != cudaSuccess) return e;
   const size_t smem_sched = 2 * (static_cast<size_t>(s.nb) + 1) * sizeof(int);
-  static bool sched_attr[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !sched_attr[dev]) {
+  static std::atomic<bool> sched_attr[64];
+  e = once_per_device(sched_attr, [] {
     const int max_dyn = 2 * (16384 + 1) * static_cast<int>(sizeof(int));
-    if ((e = cudaFuncSetAttribute(length_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  max_dyn)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  max_dyn)) != cudaSuccess)
-      return e;
-    sched_attr[dev] = true;
-  }
+    cudaError_t r = cudaFuncSetAttribute(length_hist_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                max_dyn);
+  });
+  if (e != cudaSuccess) return e;
   const size_t bins_bytes = ((static_cast<size_t>(s.nb) + 1) * 4 + 255) & ~static_cast<size_t>(255);
   int32_t* bins = static_cast<int32_t*>(scratch);
   int32_t* fill = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + bins_bytes);

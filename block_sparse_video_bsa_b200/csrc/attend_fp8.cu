@@ -481,15 +481,12 @@ cudaError_t launch_attend_fp8(const Shape& s, const AttendMapsFp8& maps, const F
                               const int32_t* idx, const float* bias, void* O, float* lse,
                               cudaStream_t st) {
   constexpr size_t smem = kOffCtl + sizeof(Ctl);
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(attend_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(attend_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem);
+  });
+  if (e != cudaSuccess) return e;
   Args a;
   a.idx = idx;
   a.bias = bias;

@@ -6,7 +6,25 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace bsa {
+
+// Runs `set` (a kernel-attribute setter) on the current device unless an
+// earlier call on that device already succeeded.  The flags are atomics, so
+// two host threads making their first call at the same time do not race; at
+// worst both run `set`, which is idempotent.
+template <class F>
+cudaError_t once_per_device(std::atomic<bool> (&done)[64], F set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return set();
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+  return e;
+}
 
 struct Shape {
   int B, H, N;      // D is fixed at 128

@@ -722,10 +722,8 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
   const size_t gram_smem = kStages * kTile + sizeof(GramSmem) + 1024;
   const size_t whiten_smem = 3 * kTile + sizeof(WhitenSmem) + 1024;
   const size_t factor_smem = 128 * 129 * sizeof(double);
-  static bool attr[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr[dev]) {
+  static std::atomic<bool> attr[64];
+  cudaError_t ea = once_per_device(attr, [&] {
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(gram_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   gram_smem)) != cudaSuccess ||
@@ -736,8 +734,9 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
         (e = cudaFuncSetAttribute(factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   factor_smem)) != cudaSuccess)
       return e;
-    attr[dev] = true;
-  }
+    return cudaSuccess;
+  });
+  if (ea != cudaSuccess) return ea;
   int32_t* pa = perm_out;
   int32_t* pb = w.perm_tmp;
   init_perm_kernel<<<dim3(64, BH), 256, 0, st>>>(pa, s.N);

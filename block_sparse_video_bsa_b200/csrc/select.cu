@@ -250,15 +250,12 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float* __restric
 template <int kPerLane, bool kThresh = false>
 cudaError_t launch_select_t(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
                             int32_t* cnt, int R, size_t smem, cudaStream_t st, float tau = 0.f) {
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel<kPerLane, kThresh>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(select_kernel<kPerLane, kThresh>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  });
+  if (e != cudaSuccess) return e;
   const dim3 grid((s.nb + R - 1) / R, s.B * s.H);
   const float scale = 0.088388347648318440550f;
   const int kcap = kThresh ? s.nb : s.kcap;

@@ -182,7 +182,10 @@ int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK,
  *     e.g. B=1, H=56, N=73,416, top_k=64).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept for the life of the
+ *     process: calling on a device after cudaDeviceReset, or from a driver
+ *     context other than the device's primary context, is not supported
+ *     (the array may then live at another address).
  *   - All calls share the one array per device and it keeps the last call's
  *     contents.  No part of it needs to start at zero (every stage fully
  *     writes what the next stage reads), but calls that overlap on the GPU

@@ -72,9 +72,14 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
     assert L.bsa_forward_host(P, a, a, a, a, None, a, a, a, None, None, a, 1 << 40,
                               None) == bsa.BSA_ERR_INVALID
     assert L.bsa_debug_expired_wait(None, 1000, None) == bsa.BSA_ERR_INVALID
-    # the mean variant does not need an anchor; the anchor variant does
+    # The mean variant does not need an anchor, the anchor variant does.  The
+    # mean-variant call passes the null-anchor check and is then stopped by a
+    # misaligned bias, so it never reaches the device even on a GPU machine.
     pm = _p(variant="mean")
-    assert L.bsa_summarize(ctypes.byref(pm), a, a, None, a, a, a, a, None) != bsa.BSA_ERR_INVALID
+    bias_odd = ctypes.c_void_p((1 << 20) + 2)
+    assert L.bsa_summarize(ctypes.byref(pm), a, a, None, a, a, a, bias_odd, None) == \
+        bsa.BSA_ERR_ALIGN
+    assert L.bsa_summarize(P, a, a, None, a, a, a, bias_odd, None) == bsa.BSA_ERR_INVALID
 
 
 def test_status_strings():
