@@ -147,9 +147,9 @@ def test_reblock_full_size_sampled_head():
     Qh, Kh, Vh = (x[:, h:h + 1].contiguous() for x in (Q, K, V))
     Qp, Kp, Vp = (torch.empty_like(Qh) for _ in range(3))
     bsa.bsa_permute(p1, Qh, Kh, Vh, perm[:, h:h + 1].contiguous(), Qp, Kp, Vp)
-    buf = run_stages(Qp, Kp, Vp, cfg["top_k"], cfg["prefix"], cfg["variant"], with_lse=False)
+    buf = run_stages(Qp, Kp, Vp, cfg["top_k"], cfg["prefix"], cfg["variant"], with_lse=True)
     check_head(buf, Qp, Kp, Vp, 0, 0, cfg["top_k"], cfg["prefix"], cfg["variant"],
-               check_lse=False)
+               check_lse=True)
     Ob = torch.empty_like(Qh)
     bsa.bsa_unpermute(p1, buf["O"], None, perm[:, h:h + 1].contiguous(), Ob)
     torch.cuda.synchronize()
