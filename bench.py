@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload h3_768p_5s] [--top-k K] [--no-cpu-baseline] [--no-e2e]
-                    [--precision bf16|fp8] [--reblock] [--tau T]
+                    [--precision bf16|fp8] [--reblock] [--tau T] [--shard heads [--gather]]
 
 One step = one whole attention call (pool -> summarize -> select -> attend,
 all through the C ABI) over one batch of synthetic bf16 input of the 768p-5s
@@ -18,9 +18,15 @@ selection keeps the key blocks at least T standard deviations above each
 row's mean score (bsa_select_threshold) and the attention runs over those
 variable-length lists (bsa_attend_lists, schedule kernels included in its
 stage time).  The default (bf16, top_k) line is the headline.
-Prints ONE JSON line on rank 0.  Multi-GPU (torchrun): every rank runs its own
-independent call on its own inputs (weak scaling, no data-path collective);
-the time is the max over ranks.
+Prints ONE JSON line on rank 0.  Multi-GPU (torchrun): the (b, h) slices of
+the job are split into contiguous per-rank ranges and every rank runs one
+attention call over its own range, with no data-path collective (every stage
+is per head).  By default the job grows with the ranks (weak scaling: the
+batch holds one video per rank, each rank runs its video's 56 heads);
+``--shard heads`` splits the heads of one video across the ranks instead
+(strong scaling: 56 / N heads per rank), and ``--gather`` then adds an
+all-gather of O over NCCL to the timed step.  The time is the max over ranks;
+the effective FLOPs are summed over ranks.
 """
 
 from __future__ import annotations
@@ -60,7 +66,13 @@ def parse_args():
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"])
     ap.add_argument("--reblock", action="store_true")
     ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--shard", default=None, choices=["heads"],
+                    help="split one call's heads across the ranks (strong scaling)")
+    ap.add_argument("--gather", action="store_true",
+                    help="with --shard heads: all-gather O over NCCL inside the timed step")
     args = ap.parse_args()
+    if args.gather and args.shard != "heads":
+        ap.error("--gather needs --shard heads")
     if args.reblock and args.precision != "bf16":
         ap.error("--reblock runs the bf16 path")
     if args.tau is not None and (args.reblock or args.precision != "bf16"):
@@ -140,6 +152,18 @@ def max_over_ranks(ms: float, device=None) -> float:
         return float(ms)
     t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    """Sum of a per-rank quantity over all ranks (identity without a process
+    group): the effective FLOPs of the ranks' head ranges."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
 
@@ -306,6 +330,15 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+def parallelism_label(args, world, total_bh, nbh, gather):
+    """How the job's (b, h) slices are split over the ranks."""
+    if args.shard == "heads":
+        return (f"heads of one call split over {world} GPU(s): {total_bh} heads, {nbh} on rank 0, "
+                f"no collective in the forward" + ("; O all-gathered over NCCL" if gather else ""))
+    return (f"one video per GPU: B={world} x {total_bh // max(world, 1)} heads, each rank runs "
+            f"its own video's heads, no data-path collective")
+
+
 def data_label(cfg):
     """What the timed inputs are: the seeded generator kind and the workload shape."""
     kind = {"block_offset": "per-block-offset", "iid": "iid N(0,1)"}.get(cfg["kind"], cfg["kind"])
@@ -313,11 +346,13 @@ def data_label(cfg):
             f"H={cfg['H']}, N={cfg['N']})")
 
 
-def config_block(cfg, **extra):
+def config_block(cfg, local_bh=None, **extra):
+    """The workload's sizes; ``local_bh`` = (b, h) slices one rank runs."""
+    bh = cfg["B"] * cfg["H"] if local_bh is None else local_bh
     d = {"workload": cfg["name"], "B": cfg["B"], "H": cfg["H"], "N": cfg["N"], "d": 128,
          "top_k": cfg["top_k"], "prefix": cfg["prefix"], "summary": cfg["variant"],
          "inputs": cfg["kind"], "l2": "inputs larger than L2 (Q+K+V = "
-         f"{3 * cfg['B'] * cfg['H'] * cfg['N'] * 256 / 1e9:.2f} GB per step)"}
+         f"{3 * bh * cfg['N'] * 256 / 1e9:.2f} GB per step and GPU)"}
     d.update(extra)
     return d
 
@@ -340,7 +375,8 @@ def main():
     import torch
     import torch.distributed as dist
     from block_sparse_video_bsa_b200 import bsa
-    from block_sparse_video_bsa_b200.inputs import make_qkv
+    from block_sparse_video_bsa_b200.inputs import make_qkv_slices
+    from block_sparse_video_bsa_b200.shard import gather_heads, head_range
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -351,9 +387,18 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
-    B, H, N = cfg["B"], cfg["H"], cfg["N"]
+    # This rank's contiguous range of the job's (b, h) slices, run as one
+    # sub-call with B = 1 and H = the range's length.
+    N = cfg["N"]
     top_k, prefix, variant = cfg["top_k"], cfg["prefix"], cfg["variant"]
-    Q, K, V = make_qkv(B, H, N, 128, cfg["kind"], seed=rank, device=dev)
+    B_job = cfg["B"] * (1 if args.shard == "heads" else world)
+    total_bh = B_job * cfg["H"]
+    bh0, nbh = head_range(total_bh, world, rank)
+    if nbh == 0:
+        raise SystemExit(f"rank {rank}: no heads to run ({total_bh} slices over {world} ranks)")
+    Q, K, V = make_qkv_slices(B_job, cfg["H"], N, bh0, nbh, 128, cfg["kind"], seed=0, device=dev)
+    B, H = 1, nbh
+    gather = args.gather and world > 1
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     p = bsa.params(B, H, N, top_k, prefix, variant, dev_status=status)
     buf = bsa.stage_buffers(B, H, N, top_k, prefix, variant, device=dev)
@@ -378,7 +423,8 @@ def main():
     else:
         Qa, Ka, Va, Oa = Q, K, V, O
     names = (["reblock", "permute"] if rbl else []) + ["pool", "summarize", "select"] + \
-        (["quantize"] if fp8 else []) + ["attend"] + (["unpermute"] if rbl else [])
+        (["quantize"] if fp8 else []) + ["attend"] + (["unpermute"] if rbl else []) + \
+        (["gather"] if gather else [])
     nev = len(names) + 1
 
     def step(ev=None):
@@ -418,15 +464,18 @@ def main():
         if rbl:
             bsa.bsa_unpermute(p, Oa, None, perm, O, None, stream)
             mark()
+        if gather:   # every rank ends the step holding the whole O
+            gather_heads(O, total_bh)
+            mark()
 
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize(dev)
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {bsa.status_string(int(status.item()))}")
-    pairs = effective_pairs(buf["idx"].cpu().numpy(), buf["cnt"].cpu().numpy(), N, prefix) \
-        * 1  # all B*H heads
-    flops_step = 4 * 128 * pairs
+    pairs = effective_pairs(buf["idx"].cpu().numpy(), buf["cnt"].cpu().numpy(), N, prefix)
+    flops_step = 4 * 128 * pairs               # this rank's heads
+    flops_job = sum_over_ranks(flops_step, dev)  # every rank's heads
     nb = bsa.bsa_num_blocks(p)
     mean_kept = None
     if thr:   # video blocks kept per video query block, over all heads
@@ -455,7 +504,7 @@ def main():
                 for i in range(nev - 1)]
     total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
-    value = job_tflops(flops_step, args.steps, world, total_ms)
+    value = job_tflops(flops_job, args.steps, 1, total_ms)
 
     # end to end through the C ABI from pinned host buffers
     e2e = None
@@ -500,7 +549,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
-        e2e = {"value": job_tflops(flops_step, args.e2e_steps, world, e_ms),
+        e2e = {"value": job_tflops(flops_job, args.e2e_steps, 1, e_ms),
                "unit": "TFLOP/s", "ms_per_call": e_ms / args.e2e_steps,
                "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                "d2h_bytes_per_step": O.numel() * O.element_size(),
@@ -522,7 +571,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
-        e2e = {"value": job_tflops(flops_step, args.e2e_steps, world, e_ms),
+        e2e = {"value": job_tflops(flops_job, args.e2e_steps, 1, e_ms),
                "unit": "TFLOP/s", "ms_per_call": e_ms / args.e2e_steps,
                "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                "d2h_bytes_per_step": O.numel() * O.element_size(),
@@ -539,7 +588,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        hh = [0, 1, 2]
+        hh = list(range(min(3, H)))
         Qh = [Q[0, h].double().cpu().numpy() for h in hh]
         Kh = [K[0, h].double().cpu().numpy() for h in hh]
         Vh = [V[0, h].double().cpu().numpy() for h in hh]
@@ -549,16 +598,20 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True,
+            "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None,
             "dtype": "e4m3" if fp8 else "bf16",
             "data": data_label(cfg),
-            "config": config_block(cfg, parallelism=f"{world} independent calls (one per GPU)",
+            "config": config_block(cfg, local_bh=nbh,
+                                   parallelism=parallelism_label(args, world, total_bh, nbh,
+                                                                 gather),
+                                   global_batch=B_job, heads_per_rank=nbh,
                                    **({"layout": "adaptive reblocking (q_reuse_k)"} if rbl
                                       else {}),
                                    **({"selection": f"threshold tau={args.tau}",
                                        "mean_kept_blocks": mean_kept} if thr else {})),
             "ms_per_call": ms_per_step,
-            "effective_tflop_per_call": flops_step / 1e12,
+            "effective_tflop_per_call": flops_job / 1e12,
             "stages_ms": dict(zip(names, stage_ms)),
             "roofline": {"kernel": "attend_fp8_kernel" if fp8 else "attend_kernel",
                          "bound": "tensor", "achieved": attend_tflops,

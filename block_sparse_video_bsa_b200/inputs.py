@@ -63,6 +63,24 @@ def make_qkv(B: int, H: int, N: int, d: int = 128, kind: str = "iid", seed: int 
     return tuple(make_tensor(t, B, H, N, d, kind, seed, device) for t in ("q", "k", "v"))
 
 
+def make_qkv_slices(B: int, H: int, N: int, start: int, count: int, d: int = 128,
+                    kind: str = "iid", seed: int = 0, device="cpu"):
+    """(Q, K, V) slices start .. start+count-1 (in (b, h) order) of the tensors
+    ``make_qkv(B, H, N, ...)`` builds, each as a contiguous bf16
+    [1, count, N, d] tensor: a rank regenerates only the heads it owns, bit
+    for bit equal to the same slices of the whole tensors."""
+    out = []
+    for t in ("q", "k", "v"):
+        x = torch.empty(1, count, N, d, dtype=torch.bfloat16, device=device)
+        gen = torch.Generator(device=device)
+        for i in range(count):
+            b, h = divmod(start + i, H)
+            gen.manual_seed(slice_seed(seed, t, b, h, H))
+            x[0, i] = _one_slice(N, d, kind, gen, device)
+        out.append(x)
+    return tuple(out)
+
+
 # The five workloads: shapes of the pages' "Measured" table (56 heads,
 # head_dim 128, H3's 24 fps sequence lengths) plus a small iid case.
 CONFIGS = {

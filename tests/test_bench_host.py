@@ -52,7 +52,9 @@ def _rank_main(rank, world, port, out_q):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     local_ms = [120.0, 250.0][rank]             # rank 1 is the slow one
     m = bench.max_over_ranks(local_ms)
-    out_q.put((rank, m, bench.job_tflops(9.11e12, 10, world, m)))
+    # the ranks' head ranges carry different effective FLOPs; the job's is the sum
+    f = bench.sum_over_ranks([4.0e12, 3.0e12][rank])
+    out_q.put((rank, m, bench.job_tflops(9.11e12, 10, world, m), f))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -68,9 +70,10 @@ def test_two_rank_timing_takes_the_slowest_rank():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, m, v in res:
+    for rank, m, v, f in res:
         assert m == 250.0
         assert v == pytest.approx(2 * 9.11 * 10 / 0.25)
+        assert f == 7.0e12
 
 
 def test_max_over_ranks_without_process_group_is_identity():
@@ -103,3 +106,19 @@ def test_threshold_options():
     assert out.returncode == 0, out.stderr
     line = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
     assert line["config"]["selection"] == "threshold tau=1.0" and line["value"] > 0
+
+
+def test_shard_options():
+    # --gather only makes sense when one call's heads are split over the ranks
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gather"],
+                         capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert out.returncode != 0 and "--gather" in out.stderr
+
+
+def test_parallelism_labels_name_the_split():
+    class A:
+        shard = "heads"
+    assert "7 on rank 0" in bench.parallelism_label(A, 8, 56, 7, False)
+    assert "all-gathered" in bench.parallelism_label(A, 8, 56, 7, True)
+    A.shard = None
+    assert "B=8 x 56 heads" in bench.parallelism_label(A, 8, 448, 56, False)
