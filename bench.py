@@ -2,7 +2,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload h3_768p_5s] [--top-k K] [--no-cpu-baseline] [--no-e2e]
-                    [--precision bf16|fp8] [--reblock] [--tau T] [--shard heads [--gather]]
+                    [--precision bf16|fp8] [--reblock] [--tau T] [--extra-tokens N]
+                    [--shard heads [--gather]]
 
 One step = one whole attention call (pool -> summarize -> select -> attend,
 all through the C ABI) over one batch of synthetic bf16 input of the 768p-5s
@@ -17,7 +18,11 @@ tensor ratio (2).  ``--tau T`` times the threshold-selection option: the
 selection keeps the key blocks at least T standard deviations above each
 row's mean score (bsa_select_threshold) and the attention runs over those
 variable-length lists (bsa_attend_lists, schedule kernels included in its
-stage time).  The default (bf16, top_k) line is the headline.
+stage time).  ``--extra-tokens N`` times the extra-token option: the N
+top-scoring tokens of the unlisted blocks of every query block are read
+exactly (bsa_select_extra), the blocks that lose tokens get summary rows of
+their remaining tokens (bsa_extra_summaries) and the attention reads both
+(bsa_attend_extra).  The default (bf16, top_k) line is the headline.
 Prints ONE JSON line on rank 0.  Multi-GPU (torchrun): the (b, h) slices of
 the job are split into contiguous per-rank ranges and every rank runs one
 attention call over its own range, with no data-path collective (every stage
@@ -66,6 +71,7 @@ def parse_args():
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"])
     ap.add_argument("--reblock", action="store_true")
     ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--extra-tokens", type=int, default=None)
     ap.add_argument("--shard", default=None, choices=["heads"],
                     help="split one call's heads across the ranks (strong scaling)")
     ap.add_argument("--gather", action="store_true",
@@ -77,6 +83,11 @@ def parse_args():
         ap.error("--reblock runs the bf16 path")
     if args.tau is not None and (args.reblock or args.precision != "bf16"):
         ap.error("--tau runs the bf16 path without reblocking")
+    if args.extra_tokens is not None and (args.reblock or args.precision != "bf16" or
+                                          args.tau is not None):
+        ap.error("--extra-tokens runs the bf16 top-k path without reblocking")
+    if args.extra_tokens is not None and not (0 <= args.extra_tokens <= 512):
+        ap.error("--extra-tokens takes 0 .. 512")
     return args
 
 
@@ -128,6 +139,31 @@ def effective_pairs(idx, cnt, N, prefix):
     valid = np.arange(idx.shape[-1])[None, None, :] < cnt[:, :, None]
     exact = np.where(valid, sizes[np.clip(idx, 0, nb - 1)], 0).sum(-1)
     summ = np.where(np.arange(nb)[None, :] >= pb, (nb - pb) - (cnt - pb), 0)
+    return int((sizes[None, :] * (exact + summ)).sum())
+
+
+def effective_pairs_extra(idx, cnt, extra, ecnt, side_cnt, N, prefix):
+    """Computed pairs of the extra-token path (all heads): exact pairs over the
+    listed blocks' real tokens and the extra tokens, plus one summary column
+    per unlisted video block that holds none of the row's extra tokens and one
+    per side summary row, for every video query row."""
+    sizes = block_sizes(N)
+    nb = len(sizes)
+    pb = prefix // 128
+    idx = idx.reshape(-1, nb, idx.shape[-1])
+    cnt = cnt.reshape(-1, nb)
+    extra = extra.reshape(-1, nb, extra.shape[-1])
+    ecnt = ecnt.reshape(-1, nb)
+    side_cnt = side_cnt.reshape(-1, nb)
+    valid = np.arange(idx.shape[-1])[None, None, :] < cnt[:, :, None]
+    exact = np.where(valid, sizes[np.clip(idx, 0, nb - 1)], 0).sum(-1) + ecnt
+    ev = np.arange(extra.shape[-1])[None, None, :] < ecnt[:, :, None]
+    blk = np.where(ev, extra // 128, -1)
+    starts = ev & np.concatenate([np.ones_like(blk[..., :1], dtype=bool),
+                                  blk[..., 1:] != blk[..., :-1]], axis=-1)
+    affected = starts.sum(-1)
+    summ = np.where(np.arange(nb)[None, :] >= pb,
+                    (nb - pb) - (cnt - pb) - affected + side_cnt, 0)
     return int((sizes[None, :] * (exact + summ)).sum())
 
 
@@ -234,12 +270,42 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle
 
+def oracle_pairs(N, out, pb, query_blocks=None):
+    """Computed pairs of one oracle head (extra tokens included when the
+    output holds them): exact pairs over the listed blocks' real tokens and
+    the extra tokens, one summary column per unlisted video block that keeps
+    at least one token out of the extra ones."""
+    import oracle as orc
+    extras = out.get("extras")
+    if extras is None:
+        return orc.effective_pairs(N, out["lists"], pb, query_blocks=query_blocks)
+    bounds = orc.block_bounds(N)
+    nb = len(bounds)
+    total = 0
+    for i, (a, b) in enumerate(bounds):
+        if query_blocks is not None and i not in query_blocks:
+            continue
+        listed = set(int(j) for j in out["lists"][i])
+        exact = sum(bounds[j][1] - bounds[j][0] for j in listed) + len(extras[i])
+        summ = 0
+        if i >= pb:
+            taken = {}
+            for u in extras[i]:
+                taken[int(u) // 128] = taken.get(int(u) // 128, 0) + 1
+            summ = sum(1 for j in range(pb, nb) if j not in listed and
+                       taken.get(j, 0) < bounds[j][1] - bounds[j][0])
+        total += (b - a) * (exact + summ)
+    return total
+
+
 def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False, reblock=False,
-                tau=None):
+                tau=None, extra_tokens=None):
     """The fp64 oracle as it stands, on whole heads, until ~budget_s of CPU work
     (the FP8 oracle for ``fp8``, the reblocking oracle for ``reblock``, the
-    threshold oracle when ``tau`` is given)."""
+    threshold oracle when ``tau`` is given, the extra-token oracle when
+    ``extra_tokens`` is)."""
     import oracle as orc
+    from oracle import bsa_oracle_extra as orcx
     from oracle import bsa_oracle_fp8 as orc8
     from oracle import bsa_oracle_reblock as orcr
     from oracle import bsa_oracle_threshold as orct
@@ -248,6 +314,9 @@ def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False, reblock=
     sel = cfg["top_k"]
     if tau is not None:
         head_fn, sel = orct.forward_head_threshold, tau
+    if extra_tokens is not None:
+        def head_fn(Q_, K_, V_, top_k_, prefix_, variant_):
+            return orcx.forward_head_extra(Q_, K_, V_, top_k_, extra_tokens, prefix_, variant_)
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
@@ -258,7 +327,7 @@ def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False, reblock=
     heads = 0
     for h in range(min(max_heads, len(Qh))):
         out = head_fn(Qh[h], Kh[h], Vh[h], sel, cfg["prefix"], cfg["variant"])
-        pairs += orc.effective_pairs(len(Qh[h]), out["lists"], cfg["prefix"] // 128)
+        pairs += oracle_pairs(len(Qh[h]), out, cfg["prefix"] // 128)
         heads += 1
         if time.perf_counter() - t0 > budget_s:
             break
@@ -267,7 +336,8 @@ def time_oracle(Qh, Kh, Vh, cfg, budget_s=20.0, max_heads=3, fp8=False, reblock=
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{heads} of {cfg['H']} heads of the workload, whole "
                       f"{'FP8 ' if fp8 else ''}{'reblocked ' if reblock else ''}"
-                      f"{'threshold ' if tau is not None else ''}path per head "
+                      f"{'threshold ' if tau is not None else ''}"
+                      f"{'extra-token ' if extra_tokens is not None else ''}path per head "
                       f"(numpy fp64, BLAS threads = {cores}); {dt:.1f} s, "
                       f"{dt / heads:.2f} s/head"}, dt / heads
 
@@ -292,7 +362,12 @@ def run_reference(args, cfg):
     times, pairs_l = [], []
     for s in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        if args.tau is None:
+        if args.extra_tokens is not None:
+            from oracle import bsa_oracle_extra as orcx
+            out = orcx.forward_head_extra(heads[0], heads[1], heads[2], cfg["top_k"],
+                                          args.extra_tokens, cfg["prefix"], cfg["variant"],
+                                          query_blocks=qblocks)
+        elif args.tau is None:
             out = orc.forward_head(heads[0], heads[1], heads[2], cfg["top_k"], cfg["prefix"],
                                    cfg["variant"], query_blocks=qblocks)
         else:
@@ -303,7 +378,7 @@ def run_reference(args, cfg):
         dt = time.perf_counter() - t0
         if s >= args.warmup:
             times.append(dt)
-            pairs_l.append(orc.effective_pairs(N, out["lists"], pb, query_blocks=qblocks))
+            pairs_l.append(oracle_pairs(N, out, pb, query_blocks=qblocks))
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
@@ -321,7 +396,9 @@ def run_reference(args, cfg):
         "data": "synthetic",
         "config": config_block(cfg, sample=sample,
                                **({"selection": f"threshold tau={args.tau}"}
-                                  if args.tau is not None else {})),
+                                  if args.tau is not None else {}),
+                               **({"extra_tokens": args.extra_tokens}
+                                  if args.extra_tokens is not None else {})),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -407,6 +484,10 @@ def main():
     fp8 = args.precision == "fp8"
     rbl = args.reblock
     thr = args.tau is not None
+    xtr = args.extra_tokens is not None
+    if xtr:
+        n_extra = args.extra_tokens
+        buf.update(bsa.extra_buffers(B, H, N, top_k, n_extra, prefix, variant, device=dev))
     if thr:
         nb0 = bsa.bsa_num_blocks(p)
         buf["idx"] = torch.empty(B, H, nb0, bsa.bsa_threshold_capacity(p), dtype=torch.int32,
@@ -423,8 +504,8 @@ def main():
     else:
         Qa, Ka, Va, Oa = Q, K, V, O
     names = (["reblock", "permute"] if rbl else []) + ["pool", "summarize", "select"] + \
-        (["quantize"] if fp8 else []) + ["attend"] + (["unpermute"] if rbl else []) + \
-        (["gather"] if gather else [])
+        (["quantize"] if fp8 else []) + (["select_extra", "extra_summaries"] if xtr else []) + \
+        ["attend"] + (["unpermute"] if rbl else []) + (["gather"] if gather else [])
     nev = len(names) + 1
 
     def step(ev=None):
@@ -441,8 +522,13 @@ def main():
             mark()
         bsa.bsa_pool(p, Qa, buf["qpool"], buf["anchor"], stream)
         mark()
-        bsa.bsa_summarize(p, Ka, Va, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"],
-                          buf["bias"], stream)
+        if xtr:
+            bsa.bsa_summarize_stats(p, K, V, buf["anchor"], buf["kpool"], buf["ksum"],
+                                    buf["vsum"], buf["bias"], buf["kstat"], buf["vstat"],
+                                    buf["lse_blk"], stream)
+        else:
+            bsa.bsa_summarize(p, Ka, Va, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"],
+                              buf["bias"], stream)
         mark()
         if thr:
             bsa.bsa_select_threshold(p, args.tau, buf["qpool"], buf["kpool"], buf["idx"],
@@ -450,7 +536,20 @@ def main():
         else:
             bsa.bsa_select(p, buf["qpool"], buf["kpool"], buf["idx"], buf["cnt"], stream)
         mark()
-        if fp8:
+        if xtr:
+            bsa.bsa_select_extra(p, n_extra, buf["qpool"], K, buf["idx"], buf["cnt"],
+                                 buf["extra"], buf["ecnt"], buf["cand"], stream)
+            mark()
+            bsa.bsa_extra_summaries(p, n_extra, K, V, buf["anchor"], buf["kpool"], buf["kstat"],
+                                    buf["vstat"], buf["lse_blk"], buf["extra"], buf["ecnt"],
+                                    buf["side_k"], buf["side_v"], buf["side_bias"],
+                                    buf["side_blk"], buf["side_cnt"], stream)
+            mark()
+            bsa.bsa_attend_extra(p, n_extra, Q, K, V, buf["idx"], buf["cnt"], buf["extra"],
+                                 buf["ecnt"], buf["ksum"], buf["vsum"], buf["bias"],
+                                 buf["side_k"], buf["side_v"], buf["side_bias"],
+                                 buf["side_cnt"], O, None, stream)
+        elif fp8:
             bsa.bsa_quantize_fp8(p, Q, K, V, buf["ksum"], buf["vsum"], ops, stream)
             mark()
             bsa.bsa_attend_fp8(p, ops, buf["idx"], buf["cnt"], buf["bias"], O, None, stream)
@@ -473,7 +572,12 @@ def main():
     torch.cuda.synchronize(dev)
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {bsa.status_string(int(status.item()))}")
-    pairs = effective_pairs(buf["idx"].cpu().numpy(), buf["cnt"].cpu().numpy(), N, prefix)
+    if xtr:
+        pairs = effective_pairs_extra(buf["idx"].cpu().numpy(), buf["cnt"].cpu().numpy(),
+                                      buf["extra"].cpu().numpy(), buf["ecnt"].cpu().numpy(),
+                                      buf["side_cnt"].cpu().numpy(), N, prefix)
+    else:
+        pairs = effective_pairs(buf["idx"].cpu().numpy(), buf["cnt"].cpu().numpy(), N, prefix)
     flops_step = 4 * 128 * pairs               # this rank's heads
     flops_job = sum_over_ranks(flops_step, dev)  # every rank's heads
     nb = bsa.bsa_num_blocks(p)
@@ -508,35 +612,41 @@ def main():
 
     # end to end through the C ABI from pinned host buffers
     e2e = None
-    if not args.no_e2e and (fp8 or rbl or thr):
-        # the public call from pinned host buffers: copies in, forward_fp8 /
-        # forward_reblock / forward_threshold, O copied back, all inside the
-        # timed region
+    if not args.no_e2e and (fp8 or rbl or thr or xtr):
+        # the option's public host-buffer call: copies in, its forward, O copied
+        # back, pipelined over chunks of heads, all inside the timed region
         hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
         hO = torch.empty_like(hQ).pin_memory()
         if fp8:
             ws8 = torch.empty(bsa.bsa_forward_fp8_workspace_bytes(p), dtype=torch.uint8,
                               device=dev)
-            fwd, fwd_name = bsa.bsa_forward_fp8, "bsa_forward_fp8"
+            fwd, fwd_name = bsa.bsa_forward_fp8_host, "bsa_forward_fp8_host"
+        elif xtr:
+            for k_ in ("kstat", "vstat", "extra", "side_k", "side_v", "side_bias", "side_blk",
+                       "cand"):
+                del buf[k_]
+            torch.cuda.empty_cache()
+            ws8 = torch.empty(bsa.bsa_forward_extra_workspace_bytes(p, n_extra),
+                              dtype=torch.uint8, device=dev)
+
+            def fwd(p_, *rest):
+                bsa.bsa_forward_extra_host(p_, n_extra, *rest)
+            fwd_name = "bsa_forward_extra_host"
         elif thr:
             ws8 = torch.empty(bsa.bsa_forward_threshold_workspace_bytes(p), dtype=torch.uint8,
                               device=dev)
 
-            def fwd(p_, Q_, K_, V_, O_, lse_, ws_, st_):
-                bsa.bsa_forward_threshold(p_, args.tau, Q_, K_, V_, O_, lse_, ws_, st_)
-            fwd_name = "bsa_forward_threshold"
+            def fwd(p_, *rest):
+                bsa.bsa_forward_threshold_host(p_, args.tau, *rest)
+            fwd_name = "bsa_forward_threshold_host"
         else:
             del Qa, Ka, Va, Oa, rb_ws
             ws8 = torch.empty(bsa.bsa_forward_reblock_workspace_bytes(p), dtype=torch.uint8,
                               device=dev)
-            fwd, fwd_name = bsa.bsa_forward_reblock, "bsa_forward_reblock"
+            fwd, fwd_name = bsa.bsa_forward_reblock_host, "bsa_forward_reblock_host"
 
         def e2e_call():
-            Q.copy_(hQ, non_blocking=True)
-            K.copy_(hK, non_blocking=True)
-            V.copy_(hV, non_blocking=True)
-            fwd(p, Q, K, V, O, None, ws8, stream)
-            hO.copy_(O, non_blocking=True)
+            fwd(p, hQ, hK, hV, hO, None, Q, K, V, O, None, ws8, stream)
         for _ in range(2):
             e2e_call()
         torch.cuda.synchronize(dev)
@@ -553,7 +663,8 @@ def main():
                "unit": "TFLOP/s", "ms_per_call": e_ms / args.e2e_steps,
                "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                "d2h_bytes_per_step": O.numel() * O.element_size(),
-               "path": f"{fwd_name} with pinned-host copies in and out (one stream)"}
+               "path": f"{fwd_name} (pinned host Q/K/V -> device -> host O, pipelined over "
+                       "chunks of heads)"}
         del hQ, hK, hV, hO, ws8
     elif not args.no_e2e:
         hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
@@ -583,6 +694,8 @@ def main():
     attend_tflops = flops_step / (attend_ms / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"]) * (2.0 if fp8 else 1.0)
     pool_bytes = stage_bytes(B, H, N, nb, bsa.bsa_select_capacity(p))
+    if xtr:   # summarize also writes the fp32 statistics of the side summaries
+        pool_bytes += B * H * nb * (512 + 512 + 4)
     pool_gbs = pool_bytes / ((stage_ms[names.index("pool")] + stage_ms[names.index("summarize")])
                              / 1e3) / 1e9
 
@@ -592,7 +705,8 @@ def main():
         Qh = [Q[0, h].double().cpu().numpy() for h in hh]
         Kh = [K[0, h].double().cpu().numpy() for h in hh]
         Vh = [V[0, h].double().cpu().numpy() for h in hh]
-        cpu, _ = time_oracle(Qh, Kh, Vh, cfg, fp8=fp8, reblock=rbl, tau=args.tau)
+        cpu, _ = time_oracle(Qh, Kh, Vh, cfg, fp8=fp8, reblock=rbl, tau=args.tau,
+                             extra_tokens=args.extra_tokens)
 
     if rank == 0:
         line = {
@@ -609,16 +723,19 @@ def main():
                                    **({"layout": "adaptive reblocking (q_reuse_k)"} if rbl
                                       else {}),
                                    **({"selection": f"threshold tau={args.tau}",
-                                       "mean_kept_blocks": mean_kept} if thr else {})),
+                                       "mean_kept_blocks": mean_kept} if thr else {}),
+                                   **({"extra_tokens": args.extra_tokens} if xtr else {})),
             "ms_per_call": ms_per_step,
             "effective_tflop_per_call": flops_job / 1e12,
             "stages_ms": dict(zip(names, stage_ms)),
-            "roofline": {"kernel": "attend_fp8_kernel" if fp8 else "attend_kernel",
+            "roofline": {"kernel": "attend_fp8_kernel" if fp8 else
+                         ("attend_kernel (extra tokens)" if xtr else "attend_kernel"),
                          "bound": "tensor", "achieved": attend_tflops,
                          "peak": peak, "unit": "TFLOP/s", "frac": attend_tflops / peak,
                          "peak_source": f"{peak_src} bf16 burst"
                                         + (" x 2 (nominal e4m3/bf16 ratio)" if fp8 else ""),
-                         "traffic": read_traffic(cfg, "attend_fp8" if fp8 else "attend"),
+                         "traffic": None if (xtr or thr or rbl) else
+                         read_traffic(cfg, "attend_fp8" if fp8 else "attend"),
                          # the same kernel against the power-capped seconds-long
                          # cuBLAS figure (the timed region is ~0.5 s of back-to-back calls)
                          "frac_sustained": attend_tflops / (float(peaks.get(
@@ -630,7 +747,8 @@ def main():
                              "bytes_per_call": pool_bytes},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": ((11 if fp8 else (7 if thr else 5))
+            "gpu_launches": ((11 if fp8 else (6 if thr else
+                                              (5 + (2 if args.extra_tokens else 0) if xtr else 5)))
                              + (reblock_launches(N, prefix) + 2 if rbl else 0)) * args.steps,
             "clocks": clock_info,
             "context": {"pages_rtx_pro_6000_sparse_ms": 30.7 if cfg["N"] == 37_740 else None},

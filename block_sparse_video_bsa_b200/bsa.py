@@ -88,7 +88,21 @@ _SIGS = {
     "bsa_forward_threshold_workspace_bytes": (ctypes.c_size_t, [_P]),
     "bsa_forward_threshold": (ctypes.c_int, [_P, ctypes.c_float, _vp, _vp, _vp, _vp, _vp, _vp,
                                              ctypes.c_size_t, _vp]),
+    "bsa_extra_side_capacity": (ctypes.c_int32, [_P, ctypes.c_int32]),
+    "bsa_summarize_stats": (ctypes.c_int, [_P] + [_vp] * 11),
+    "bsa_select_extra_workspace_bytes": (ctypes.c_size_t, [_P, ctypes.c_int32]),
+    "bsa_select_extra": (ctypes.c_int, [_P, ctypes.c_int32] + [_vp] * 7 + [ctypes.c_size_t, _vp]),
+    "bsa_extra_summaries": (ctypes.c_int, [_P, ctypes.c_int32] + [_vp] * 15),
+    "bsa_attend_extra": (ctypes.c_int, [_P, ctypes.c_int32] + [_vp] * 17),
+    "bsa_forward_extra_workspace_bytes": (ctypes.c_size_t, [_P, ctypes.c_int32]),
+    "bsa_forward_extra": (ctypes.c_int, [_P, ctypes.c_int32] + [_vp] * 6 + [ctypes.c_size_t, _vp]),
 }
+_HOST12 = [_vp] * 11 + [ctypes.c_size_t, _vp]
+_SIGS["bsa_forward_fp8_host"] = (ctypes.c_int, [_P] + _HOST12)
+_SIGS["bsa_forward_threshold_host"] = (ctypes.c_int, [_P, ctypes.c_float] + _HOST12)
+_SIGS["bsa_forward_extra_host"] = (ctypes.c_int, [_P, ctypes.c_int32] + _HOST12)
+_SIGS["bsa_forward_reblock_host"] = (ctypes.c_int, [_P] + _HOST12)
+BSA_MAX_EXTRA_TOKENS = 512
 
 
 def lib() -> ctypes.CDLL:
@@ -187,6 +201,37 @@ def bsa_forward_host(p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, s
                                   _ptr(hlse), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dO), _ptr(dlse),
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream)), "bsa_forward_host")
+
+
+def _host_args(hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, stream):
+    return (_ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hO), _ptr(hlse), _ptr(dQ), _ptr(dK), _ptr(dV),
+            _ptr(dO), _ptr(dlse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream))
+
+
+def bsa_forward_fp8_host(p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, stream=None):
+    _check(lib().bsa_forward_fp8_host(ctypes.byref(p), *_host_args(
+        hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, stream)), "bsa_forward_fp8_host")
+
+
+def bsa_forward_threshold_host(p, tau, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace,
+                               stream=None):
+    _check(lib().bsa_forward_threshold_host(ctypes.byref(p), float(tau), *_host_args(
+        hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, stream)),
+        "bsa_forward_threshold_host")
+
+
+def bsa_forward_extra_host(p, n_extra, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace,
+                           stream=None):
+    _check(lib().bsa_forward_extra_host(ctypes.byref(p), int(n_extra), *_host_args(
+        hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, stream)), "bsa_forward_extra_host")
+
+
+def bsa_forward_reblock_host(p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace,
+                             stream=None):
+    _check(lib().bsa_forward_reblock_host(ctypes.byref(p), *_host_args(
+        hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, stream)),
+        "bsa_forward_reblock_host")
 
 
 def bsa_forward_noalloc(p, Q, K, V, O, lse=None, stream=None):
@@ -316,6 +361,97 @@ def bsa_forward_threshold(p, tau, Q, K, V, O, lse, workspace, stream=None):
                                        _ptr(O), _ptr(lse), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(),
                                        _stream(stream)), "bsa_forward_threshold")
+
+
+def bsa_extra_side_capacity(p: bsa_params, n_extra: int) -> int:
+    return lib().bsa_extra_side_capacity(ctypes.byref(p), int(n_extra))
+
+
+def bsa_summarize_stats(p, K, V, anchor, kpool, ksum, vsum, bias, kstat, vstat, lse_blk,
+                        stream=None):
+    _check(lib().bsa_summarize_stats(ctypes.byref(p), _ptr(K), _ptr(V), _ptr(anchor), _ptr(kpool),
+                                     _ptr(ksum), _ptr(vsum), _ptr(bias), _ptr(kstat), _ptr(vstat),
+                                     _ptr(lse_blk), _stream(stream)), "bsa_summarize_stats")
+
+
+def bsa_select_extra_workspace_bytes(p: bsa_params, n_extra: int) -> int:
+    return lib().bsa_select_extra_workspace_bytes(ctypes.byref(p), int(n_extra))
+
+
+def bsa_select_extra(p, n_extra, qpool, K, idx, cnt, extra, ecnt, workspace, stream=None):
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().bsa_select_extra(ctypes.byref(p), int(n_extra), _ptr(qpool), _ptr(K), _ptr(idx),
+                                  _ptr(cnt), _ptr(extra), _ptr(ecnt), _ptr(workspace), nbytes,
+                                  _stream(stream)), "bsa_select_extra")
+
+
+def bsa_extra_summaries(p, n_extra, K, V, anchor, kpool, kstat, vstat, lse_blk, extra, ecnt,
+                        side_k, side_v, side_bias, side_blk, side_cnt, stream=None):
+    _check(lib().bsa_extra_summaries(ctypes.byref(p), int(n_extra), _ptr(K), _ptr(V), _ptr(anchor),
+                                     _ptr(kpool), _ptr(kstat), _ptr(vstat), _ptr(lse_blk),
+                                     _ptr(extra), _ptr(ecnt), _ptr(side_k), _ptr(side_v),
+                                     _ptr(side_bias), _ptr(side_blk), _ptr(side_cnt),
+                                     _stream(stream)), "bsa_extra_summaries")
+
+
+def bsa_attend_extra(p, n_extra, Q, K, V, idx, cnt, extra, ecnt, ksum, vsum, bias, side_k, side_v,
+                     side_bias, side_cnt, O, lse=None, stream=None):
+    _check(lib().bsa_attend_extra(ctypes.byref(p), int(n_extra), _ptr(Q), _ptr(K), _ptr(V),
+                                  _ptr(idx), _ptr(cnt), _ptr(extra), _ptr(ecnt), _ptr(ksum),
+                                  _ptr(vsum), _ptr(bias), _ptr(side_k), _ptr(side_v),
+                                  _ptr(side_bias), _ptr(side_cnt), _ptr(O), _ptr(lse),
+                                  _stream(stream)), "bsa_attend_extra")
+
+
+def bsa_forward_extra_workspace_bytes(p: bsa_params, n_extra: int) -> int:
+    return lib().bsa_forward_extra_workspace_bytes(ctypes.byref(p), int(n_extra))
+
+
+def bsa_forward_extra(p, n_extra, Q, K, V, O, lse, workspace, stream=None):
+    _check(lib().bsa_forward_extra(ctypes.byref(p), int(n_extra), _ptr(Q), _ptr(K), _ptr(V),
+                                   _ptr(O), _ptr(lse), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "bsa_forward_extra")
+
+
+def extra_buffers(B, H, N, top_k, n_extra, prefix=0, variant="anchor", device="cuda"):
+    """Device tensors for the extra-token stages (statistics, lists, side
+    table, candidate scratch)."""
+    p = params(B, H, N, top_k, prefix, variant)
+    nb = bsa_num_blocks(p)
+    scap = bsa_extra_side_capacity(p, n_extra)
+    if nb < 0 or scap < 0:
+        raise BsaError(BSA_ERR_INVALID, "extra_buffers")
+    f32, bf16, i32 = torch.float32, torch.bfloat16, torch.int32
+    return dict(
+        kstat=torch.empty(B, H, nb, 128, dtype=f32, device=device),
+        vstat=torch.empty(B, H, nb, 128, dtype=f32, device=device),
+        lse_blk=torch.empty(B, H, nb, dtype=f32, device=device),
+        extra=torch.empty(B, H, nb, max(n_extra, 1), dtype=i32, device=device),
+        ecnt=torch.empty(B, H, nb, dtype=i32, device=device),
+        side_k=torch.empty(B, H, nb, max(scap, 1), 128, dtype=bf16, device=device),
+        side_v=torch.empty(B, H, nb, max(scap, 1), 128, dtype=bf16, device=device),
+        side_bias=torch.empty(B, H, nb, max(scap, 1), dtype=f32, device=device),
+        side_blk=torch.empty(B, H, nb, max(scap, 1), dtype=i32, device=device),
+        side_cnt=torch.empty(B, H, nb, dtype=i32, device=device),
+        cand=torch.empty(max(256, bsa_select_extra_workspace_bytes(p, n_extra)), dtype=torch.uint8,
+                         device=device),
+    )
+
+
+def forward_extra(Q, K, V, top_k, n_extra, prefix=0, variant="anchor", return_lse=False, ws=None,
+                  stream=None):
+    """bsa_forward_extra: block-sparse attention plus n_extra top-scoring
+    tokens per query block."""
+    B, H, N, D = Q.shape
+    p = params(B, H, N, top_k, prefix, variant, D=D)
+    O = torch.empty_like(Q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=Q.device) if return_lse else None
+    if ws is None:
+        ws = torch.empty(bsa_forward_extra_workspace_bytes(p, n_extra), dtype=torch.uint8,
+                         device=Q.device)
+    bsa_forward_extra(p, n_extra, Q, K, V, O, lse, ws, stream)
+    return (O, lse) if return_lse else O
 
 
 def bsa_debug_expired_wait(dev_status, timeout_ns: int, stream=None):

@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbsa.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 SOURCES = ["api.cu", "pool_summarize.cu", "select.cu", "attend.cu", "attend_fp8.cu", "quant_fp8.cu",
-           "reblock.cu",
+           "reblock.cu", "extra.cu",
            "noalloc.cu"]
 
 NVCC_FLAGS = [

@@ -94,6 +94,22 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t BH) {
          CUDA_SUCCESS;
 }
 
+// bf16 [total_rows, 128] viewed as a 2-D tensor with a one-row box of 64
+// columns (128 bytes, one swizzle atom): the map of row gathers
+// (tile::gather4 brings four rows per instruction).
+bool make_map_rows(CUtensorMap* m, const void* base, uint64_t total_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {128, total_rows};
+  const cuuint64_t strides[1] = {128 * 2};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // uint8 (e4m3 codes) [BH, rows, 128] viewed as a 3-D tensor; box = 128
 // columns (128 bytes, one swizzle atom) x 128 rows x 1 head.
 bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t BH) {
@@ -348,9 +364,359 @@ int attend_fp8_impl(const Shape& s, const bsa::Fp8Operands& f, const int32_t* id
   return cuda_status(bsa::launch_attend_fp8(s, maps, f, idx, bias, O, lse, st));
 }
 
+// ------------------------------------------------------------ extra tokens
+
+constexpr int kMaxExtra = BSA_MAX_EXTRA_TOKENS;
+
+bool extra_valid(const Shape& s, int n_extra) {
+  if (n_extra < 0 || n_extra > kMaxExtra) return false;
+  // row coordinates of the gathers are 32-bit
+  return static_cast<int64_t>(s.B) * s.H * s.N < (static_cast<int64_t>(1) << 31);
+}
+
+// Extra-token intermediates carved from one buffer (each piece 256-byte
+// aligned): fp32 block statistics, the token lists, the side summary table
+// and the candidate buffers of the selection.
+struct ExtraWs {
+  float *kstat, *vstat, *lse_blk;
+  int32_t *extra, *ecnt;
+  void *side_k, *side_v;
+  float* side_bias;
+  int32_t *side_blk, *side_cnt;
+  void* cand;
+};
+
+size_t extra_carve(const Shape& s, int n_extra, uint8_t* base, ExtraWs* w) {
+  const size_t bh = static_cast<size_t>(s.B) * s.H;
+  const size_t blocks = bh * s.nb;
+  const size_t scap = static_cast<size_t>(bsa::extra_side_cap(s, n_extra));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += round256(bytes);
+    return p;
+  };
+  uint8_t* kstat = take(blocks * 128 * 4);
+  uint8_t* vstat = take(blocks * 128 * 4);
+  uint8_t* lse_blk = take(blocks * 4);
+  uint8_t* extra = take(blocks * static_cast<size_t>(n_extra) * 4);
+  uint8_t* ecnt = take(blocks * 4);
+  uint8_t* side_k = take(blocks * scap * 128 * 2);
+  uint8_t* side_v = take(blocks * scap * 128 * 2);
+  uint8_t* side_bias = take(blocks * scap * 4);
+  uint8_t* side_blk = take(blocks * scap * 4);
+  uint8_t* side_cnt = take(blocks * 4);
+  uint8_t* cand = take(bsa::select_extra_scratch_bytes(s, n_extra));
+  if (w) {
+    w->kstat = reinterpret_cast<float*>(kstat);
+    w->vstat = reinterpret_cast<float*>(vstat);
+    w->lse_blk = reinterpret_cast<float*>(lse_blk);
+    w->extra = reinterpret_cast<int32_t*>(extra);
+    w->ecnt = reinterpret_cast<int32_t*>(ecnt);
+    w->side_k = side_k;
+    w->side_v = side_v;
+    w->side_bias = reinterpret_cast<float*>(side_bias);
+    w->side_blk = reinterpret_cast<int32_t*>(side_blk);
+    w->side_cnt = reinterpret_cast<int32_t*>(side_cnt);
+    w->cand = cand;
+  }
+  return off;
+}
+
+int select_extra_impl(const Shape& s, int n_extra, const float* qpool, const void* K,
+                      const int32_t* idx, const int32_t* cnt, int32_t* extra, int32_t* ecnt,
+                      void* scratch, cudaStream_t st) {
+  const size_t blocks = static_cast<size_t>(s.B) * s.H * s.nb;
+  if (n_extra == 0) return cuda_status(cudaMemsetAsync(ecnt, 0, blocks * 4, st));
+  CUtensorMap tm_k;
+  if (!make_map(&tm_k, K, s.N, static_cast<uint64_t>(s.B) * s.H)) return BSA_ERR_UNSUPPORTED;
+  return cuda_status(bsa::launch_select_extra(s, n_extra, tm_k, qpool, idx, s.kcap, cnt, extra,
+                                              ecnt, scratch, st));
+}
+
+int extra_summaries_impl(const Shape& s, int n_extra, const void* K, const void* V,
+                         const float* anchor, const float* kpool, const float* kstat,
+                         const float* vstat, const float* lse_blk, const int32_t* extra,
+                         const int32_t* ecnt, void* side_k, void* side_v, float* side_bias,
+                         int32_t* side_blk, int32_t* side_cnt, cudaStream_t st) {
+  const size_t blocks = static_cast<size_t>(s.B) * s.H * s.nb;
+  // prefix query blocks have no side rows
+  cudaError_t e = cudaMemsetAsync(side_cnt, 0, blocks * 4, st);
+  if (e != cudaSuccess || n_extra == 0) return cuda_status(e);
+  return cuda_status(bsa::launch_extra_summaries(s, n_extra, K, V, anchor, kpool, kstat, vstat,
+                                                 lse_blk, extra, ecnt, side_k, side_v, side_bias,
+                                                 side_blk, side_cnt, st));
+}
+
+int attend_extra_impl(const Shape& s, int n_extra, const void* Q, const void* K, const void* V,
+                      const int32_t* idx, const int32_t* extra, const int32_t* ecnt,
+                      const void* ksum, const void* vsum, const float* bias, const void* side_k,
+                      const void* side_v, const float* side_bias, const int32_t* side_cnt,
+                      void* O, float* lse, cudaStream_t st) {
+  bsa::AttendMaps maps;
+  bsa::AttendExtraMaps xm;
+  const uint64_t bh = static_cast<uint64_t>(s.B) * s.H;
+  const int scap = bsa::extra_side_cap(s, n_extra);
+  if (!make_map(&maps.q, Q, s.N, bh) || !make_map(&maps.k, K, s.N, bh) ||
+      !make_map(&maps.v, V, s.N, bh) || !make_map(&maps.ks, ksum, s.nb, bh) ||
+      !make_map(&maps.vs, vsum, s.nb, bh) || !make_map_rows(&xm.k2, K, bh * s.N) ||
+      !make_map_rows(&xm.v2, V, bh * s.N))
+    return BSA_ERR_UNSUPPORTED;
+  if (scap > 0) {
+    const uint64_t rows = static_cast<uint64_t>(s.nb) * scap;
+    if (!make_map(&xm.sk, side_k, rows, bh) || !make_map(&xm.sv, side_v, rows, bh))
+      return BSA_ERR_UNSUPPORTED;
+  } else {   // never read: no row has side summaries
+    xm.sk = maps.ks;
+    xm.sv = maps.vs;
+  }
+  return cuda_status(bsa::launch_attend_extra(s, maps, xm, idx, extra, ecnt, n_extra, bias,
+                                              side_bias, side_cnt, scap, O, lse, st));
+}
+
+// A forward from HOST buffers, pipelined over chunks of (b, h) slices; `fwd`
+// runs the forward of one chunk (a sub-call with B = 1) on the caller's
+// stream with the caller's workspace, which a sub-call needs no more of than
+// the whole call.  Validates the pointers of the device side before the first
+// copy, so an argument error enqueues nothing.
+template <class Fwd>
+int forward_host_pipelined(const bsa_params* p, const void* hQ, const void* hK, const void* hV,
+                           void* hO, float* hlse, void* dQ, void* dK, void* dV, void* dO,
+                           float* dlse, void* workspace, size_t workspace_bytes, void* stream,
+                           Fwd fwd) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!hQ || !hK || !hV || !hO) return BSA_ERR_INVALID;
+  if (!dQ || !dK || !dV || !dO || !workspace) return BSA_ERR_INVALID;
+  if (!aligned(dQ, 16) || !aligned(dK, 16) || !aligned(dV, 16) || !aligned(dO, 16) ||
+      !aligned(workspace, 256) || (dlse && !aligned(dlse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+
+  // Pipeline over chunks of (b, h) slices (every slice is independent):
+  // host->device copies on one helper stream, the forward on the caller's
+  // stream, device->host copies on another helper stream, ordered by events.
+  // Copies of chunk c+1 overlap the forward of chunk c, and the two copy
+  // directions overlap each other.  The helper streams and events are made
+  // per call and released when their work is done; the caller's stream
+  // waits for the last copy, so synchronising it covers everything.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = s.B * s.H;
+  const int nchunk = BH < 8 ? BH : 8;
+  const int per = (BH + nchunk - 1) / nchunk;
+  const size_t slice = static_cast<size_t>(s.N) * 128 * 2;     // bytes of one (b, h) slice
+  const size_t lslice = static_cast<size_t>(s.N) * 4;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_done = nullptr, ev_in[8] = {}, ev_comp[8] = {};
+  auto cleanup = [&]() {
+    for (int c = 0; c < 8; ++c) {
+      if (ev_in[c]) cudaEventDestroy(ev_in[c]);
+      if (ev_comp[c]) cudaEventDestroy(ev_comp[c]);
+    }
+    if (ev_start) cudaEventDestroy(ev_start);
+    if (ev_done) cudaEventDestroy(ev_done);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+  };
+  bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming) == cudaSuccess;
+  for (int c = 0; ok && c < nchunk; ++c)
+    ok = cudaEventCreateWithFlags(&ev_in[c], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&ev_comp[c], cudaEventDisableTiming) == cudaSuccess;
+  // helper streams start after earlier work on the caller's stream
+  ok = ok && cudaEventRecord(ev_start, st) == cudaSuccess &&
+       cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
+  if (!ok) {
+    cleanup();
+    return BSA_ERR_CUDA;
+  }
+  auto off = [](const void* base, size_t bytes) {
+    return static_cast<const char*>(base) + bytes;
+  };
+  for (int c = 0; c < nchunk && rc == BSA_OK; ++c) {
+    const int bh0 = c * per;
+    const int nbh = (BH - bh0) < per ? (BH - bh0) : per;
+    if (nbh <= 0) break;
+    const size_t o = static_cast<size_t>(bh0) * slice, bytes = static_cast<size_t>(nbh) * slice;
+    char* q = static_cast<char*>(dQ) + o;
+    char* k = static_cast<char*>(dK) + o;
+    char* v = static_cast<char*>(dV) + o;
+    char* out = static_cast<char*>(dO) + o;
+    float* l = dlse ? dlse + static_cast<size_t>(bh0) * s.N : nullptr;
+    if (cudaMemcpyAsync(q, off(hQ, o), bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(k, off(hK, o), bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(v, off(hV, o), bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaEventRecord(ev_in[c], s_in) != cudaSuccess ||
+        cudaStreamWaitEvent(st, ev_in[c], 0) != cudaSuccess) {
+      rc = BSA_ERR_CUDA;
+      break;
+    }
+    bsa_params sub = *p;
+    sub.B = 1;
+    sub.H = nbh;
+    if ((rc = fwd(&sub, q, k, v, out, l, workspace, workspace_bytes, stream))) break;
+    if (cudaEventRecord(ev_comp[c], st) != cudaSuccess ||
+        cudaStreamWaitEvent(s_out, ev_comp[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<char*>(hO) + o, out, bytes, cudaMemcpyDeviceToHost, s_out) !=
+            cudaSuccess ||
+        (hlse && l &&
+         cudaMemcpyAsync(hlse + static_cast<size_t>(bh0) * s.N, l, nbh * lslice,
+                         cudaMemcpyDeviceToHost, s_out) != cudaSuccess)) {
+      rc = BSA_ERR_CUDA;
+      break;
+    }
+  }
+  // the caller's stream waits for the last copy back
+  if (cudaEventRecord(ev_done, s_out) != cudaSuccess || cudaStreamWaitEvent(st, ev_done, 0) != cudaSuccess)
+    rc = rc ? rc : BSA_ERR_CUDA;
+  cleanup();
+  return rc;
+}
+
 }  // namespace
 
 extern "C" {
+
+int32_t bsa_extra_side_capacity(const bsa_params* p, int32_t n_extra) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK || !extra_valid(s, n_extra)) return -1;
+  return bsa::extra_side_cap(s, n_extra);
+}
+
+int bsa_summarize_stats(const bsa_params* p, const void* K, const void* V, const float* anchor,
+                        float* kpool, void* ksum, void* vsum, float* bias, float* kstat,
+                        float* vstat, float* lse_blk, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!K || !V || !kpool || !ksum || !vsum || !bias || !kstat || !vstat || !lse_blk)
+    return BSA_ERR_INVALID;
+  if (s.variant == BSA_SUMMARY_ANCHOR && !anchor) return BSA_ERR_INVALID;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(kpool, 16) || !aligned(ksum, 16) ||
+      !aligned(vsum, 16) || !aligned(bias, 4) || (anchor && !aligned(anchor, 16)) ||
+      !aligned(kstat, 16) || !aligned(vstat, 16) || !aligned(lse_blk, 4))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return cuda_status(bsa::launch_summarize(s, K, V, anchor, kpool, ksum, vsum, bias,
+                                           static_cast<cudaStream_t>(stream), kstat, vstat,
+                                           lse_blk));
+}
+
+size_t bsa_select_extra_workspace_bytes(const bsa_params* p, int32_t n_extra) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK || !extra_valid(s, n_extra)) return 0;
+  return bsa::select_extra_scratch_bytes(s, n_extra);
+}
+
+int bsa_select_extra(const bsa_params* p, int32_t n_extra, const float* qpool, const void* K,
+                     const int32_t* idx, const int32_t* cnt, int32_t* extra, int32_t* ecnt,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!extra_valid(s, n_extra)) return BSA_ERR_INVALID;
+  if (!qpool || !K || !idx || !cnt || !ecnt || (n_extra > 0 && (!extra || !workspace)))
+    return BSA_ERR_INVALID;
+  if (workspace_bytes < bsa::select_extra_scratch_bytes(s, n_extra)) return BSA_ERR_INVALID;
+  if (!aligned(qpool, 16) || !aligned(K, 16) || !aligned(idx, 4) || !aligned(cnt, 4) ||
+      !aligned(extra, 4) || !aligned(ecnt, 4) || !aligned(workspace, 256))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return select_extra_impl(s, n_extra, qpool, K, idx, cnt, extra, ecnt, workspace,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int bsa_extra_summaries(const bsa_params* p, int32_t n_extra, const void* K, const void* V,
+                        const float* anchor, const float* kpool, const float* kstat,
+                        const float* vstat, const float* lse_blk, const int32_t* extra,
+                        const int32_t* ecnt, void* side_k, void* side_v, float* side_bias,
+                        int32_t* side_blk, int32_t* side_cnt, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!extra_valid(s, n_extra)) return BSA_ERR_INVALID;
+  if (!K || !V || !kpool || !kstat || !vstat || !lse_blk || !ecnt || !side_cnt)
+    return BSA_ERR_INVALID;
+  if (s.variant == BSA_SUMMARY_ANCHOR && !anchor) return BSA_ERR_INVALID;
+  if (n_extra > 0 && (!extra || !side_k || !side_v || !side_bias || !side_blk))
+    return BSA_ERR_INVALID;
+  if (!aligned(K, 16) || !aligned(V, 16) || (anchor && !aligned(anchor, 16)) ||
+      !aligned(kpool, 16) || !aligned(kstat, 16) || !aligned(vstat, 16) || !aligned(lse_blk, 4) ||
+      !aligned(extra, 4) || !aligned(ecnt, 4) || !aligned(side_k, 16) || !aligned(side_v, 16) ||
+      !aligned(side_bias, 4) || !aligned(side_blk, 4) || !aligned(side_cnt, 4))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return extra_summaries_impl(s, n_extra, K, V, anchor, kpool, kstat, vstat, lse_blk, extra, ecnt,
+                              side_k, side_v, side_bias, side_blk, side_cnt,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int bsa_attend_extra(const bsa_params* p, int32_t n_extra, const void* Q, const void* K,
+                     const void* V, const int32_t* idx, const int32_t* cnt, const int32_t* extra,
+                     const int32_t* ecnt, const void* ksum, const void* vsum, const float* bias,
+                     const void* side_k, const void* side_v, const float* side_bias,
+                     const int32_t* side_cnt, void* O, float* lse, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!extra_valid(s, n_extra)) return BSA_ERR_INVALID;
+  if (!Q || !K || !V || !idx || !cnt || !ecnt || !ksum || !vsum || !bias || !side_cnt || !O)
+    return BSA_ERR_INVALID;
+  if (n_extra > 0 && (!extra || !side_k || !side_v || !side_bias)) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(ksum, 16) ||
+      !aligned(vsum, 16) || !aligned(O, 16) || !aligned(idx, 4) || !aligned(cnt, 4) ||
+      !aligned(extra, 4) || !aligned(ecnt, 4) || !aligned(bias, 4) || !aligned(side_k, 16) ||
+      !aligned(side_v, 16) || !aligned(side_bias, 4) || !aligned(side_cnt, 4) ||
+      (lse && !aligned(lse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return attend_extra_impl(s, n_extra, Q, K, V, idx, extra, ecnt, ksum, vsum, bias, side_k, side_v,
+                           side_bias, side_cnt, O, lse, static_cast<cudaStream_t>(stream));
+}
+
+size_t bsa_forward_extra_workspace_bytes(const bsa_params* p, int32_t n_extra) {
+  Shape s;
+  if (shape_of(p, &s) != BSA_OK || !extra_valid(s, n_extra)) return 0;
+  return carve(s, nullptr, nullptr) + extra_carve(s, n_extra, nullptr, nullptr);
+}
+
+int bsa_forward_extra(const bsa_params* p, int32_t n_extra, const void* Q, const void* K,
+                      const void* V, void* O, float* lse, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!extra_valid(s, n_extra)) return BSA_ERR_INVALID;
+  if (!Q || !K || !V || !O || !workspace) return BSA_ERR_INVALID;
+  const size_t ws0 = carve(s, nullptr, nullptr);
+  if (workspace_bytes < ws0 + extra_carve(s, n_extra, nullptr, nullptr)) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
+      !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  Workspace w;
+  carve(s, static_cast<uint8_t*>(workspace), &w);
+  ExtraWs x;
+  extra_carve(s, n_extra, static_cast<uint8_t*>(workspace) + ws0, &x);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = pool_impl(s, Q, w.qpool, w.anchor, st))) return rc;
+  if ((rc = cuda_status(bsa::launch_summarize(s, K, V, w.anchor, w.kpool, w.ksum, w.vsum, w.bias,
+                                              st, x.kstat, x.vstat, x.lse_blk))))
+    return rc;
+  if ((rc = select_impl(s, w.qpool, w.kpool, w.idx, w.cnt, st))) return rc;
+  if ((rc = select_extra_impl(s, n_extra, w.qpool, K, w.idx, w.cnt, x.extra, x.ecnt, x.cand, st)))
+    return rc;
+  if ((rc = extra_summaries_impl(s, n_extra, K, V, w.anchor, w.kpool, x.kstat, x.vstat, x.lse_blk,
+                                 x.extra, x.ecnt, x.side_k, x.side_v, x.side_bias, x.side_blk,
+                                 x.side_cnt, st)))
+    return rc;
+  return attend_extra_impl(s, n_extra, Q, K, V, w.idx, x.extra, x.ecnt, w.ksum, w.vsum, w.bias,
+                           x.side_k, x.side_v, x.side_bias, x.side_cnt, O, lse, st);
+}
 
 size_t bsa_reblock_workspace_bytes(const bsa_params* p) {
   Shape s;
@@ -685,96 +1051,76 @@ int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK, const 
   Shape s;
   int rc = shape_of(p, &s);
   if (rc) return rc;
-  if (!hQ || !hK || !hV || !hO) return BSA_ERR_INVALID;
-  // Validate the device side before the first copy so an error enqueues nothing.
-  if (!dQ || !dK || !dV || !dO || !workspace) return BSA_ERR_INVALID;
   if (workspace_bytes < carve(s, nullptr, nullptr)) return BSA_ERR_INVALID;
-  if (!aligned(dQ, 16) || !aligned(dK, 16) || !aligned(dV, 16) || !aligned(dO, 16) ||
-      !aligned(workspace, 256) || (dlse && !aligned(dlse, 4)))
-    return BSA_ERR_ALIGN;
-  if ((rc = check_device())) return rc;
+  return forward_host_pipelined(
+      p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, workspace_bytes, stream,
+      [](const bsa_params* sub, void* q, void* k, void* v, void* o, float* l, void* ws,
+         size_t wsb, void* st) { return bsa_forward(sub, q, k, v, o, l, ws, wsb, st); });
+}
 
-  // Pipeline over chunks of (b, h) slices (every slice is independent):
-  // host->device copies on one helper stream, the forward on the caller's
-  // stream, device->host copies on another helper stream, ordered by events.
-  // Copies of chunk c+1 overlap the forward of chunk c, and the two copy
-  // directions overlap each other.  The helper streams and events are made
-  // per call and released when their work is done; the caller's stream
-  // waits for the last copy, so synchronising it covers everything.
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int BH = s.B * s.H;
-  const int nchunk = BH < 8 ? BH : 8;
-  const int per = (BH + nchunk - 1) / nchunk;
-  const size_t slice = static_cast<size_t>(s.N) * 128 * 2;     // bytes of one (b, h) slice
-  const size_t lslice = static_cast<size_t>(s.N) * 4;
-  cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t ev_start = nullptr, ev_done = nullptr, ev_in[8] = {}, ev_comp[8] = {};
-  auto cleanup = [&]() {
-    for (int c = 0; c < 8; ++c) {
-      if (ev_in[c]) cudaEventDestroy(ev_in[c]);
-      if (ev_comp[c]) cudaEventDestroy(ev_comp[c]);
-    }
-    if (ev_start) cudaEventDestroy(ev_start);
-    if (ev_done) cudaEventDestroy(ev_done);
-    if (s_in) cudaStreamDestroy(s_in);
-    if (s_out) cudaStreamDestroy(s_out);
-  };
-  bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) == cudaSuccess &&
-            cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming) == cudaSuccess;
-  for (int c = 0; ok && c < nchunk; ++c)
-    ok = cudaEventCreateWithFlags(&ev_in[c], cudaEventDisableTiming) == cudaSuccess &&
-         cudaEventCreateWithFlags(&ev_comp[c], cudaEventDisableTiming) == cudaSuccess;
-  // helper streams start after earlier work on the caller's stream
-  ok = ok && cudaEventRecord(ev_start, st) == cudaSuccess &&
-       cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
-       cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
-  if (!ok) {
-    cleanup();
-    return BSA_ERR_CUDA;
-  }
-  auto off = [](const void* base, size_t bytes) {
-    return static_cast<const char*>(base) + bytes;
-  };
-  for (int c = 0; c < nchunk && rc == BSA_OK; ++c) {
-    const int bh0 = c * per;
-    const int nbh = (BH - bh0) < per ? (BH - bh0) : per;
-    if (nbh <= 0) break;
-    const size_t o = static_cast<size_t>(bh0) * slice, bytes = static_cast<size_t>(nbh) * slice;
-    char* q = static_cast<char*>(dQ) + o;
-    char* k = static_cast<char*>(dK) + o;
-    char* v = static_cast<char*>(dV) + o;
-    char* out = static_cast<char*>(dO) + o;
-    float* l = dlse ? dlse + static_cast<size_t>(bh0) * s.N : nullptr;
-    if (cudaMemcpyAsync(q, off(hQ, o), bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-        cudaMemcpyAsync(k, off(hK, o), bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-        cudaMemcpyAsync(v, off(hV, o), bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-        cudaEventRecord(ev_in[c], s_in) != cudaSuccess ||
-        cudaStreamWaitEvent(st, ev_in[c], 0) != cudaSuccess) {
-      rc = BSA_ERR_CUDA;
-      break;
-    }
-    bsa_params sub = *p;
-    sub.B = 1;
-    sub.H = nbh;
-    if ((rc = bsa_forward(&sub, q, k, v, out, l, workspace, workspace_bytes, stream))) break;
-    if (cudaEventRecord(ev_comp[c], st) != cudaSuccess ||
-        cudaStreamWaitEvent(s_out, ev_comp[c], 0) != cudaSuccess ||
-        cudaMemcpyAsync(static_cast<char*>(hO) + o, out, bytes, cudaMemcpyDeviceToHost, s_out) !=
-            cudaSuccess ||
-        (hlse && l &&
-         cudaMemcpyAsync(hlse + static_cast<size_t>(bh0) * s.N, l, nbh * lslice,
-                         cudaMemcpyDeviceToHost, s_out) != cudaSuccess)) {
-      rc = BSA_ERR_CUDA;
-      break;
-    }
-  }
-  // the caller's stream waits for the last copy back
-  if (cudaEventRecord(ev_done, s_out) != cudaSuccess || cudaStreamWaitEvent(st, ev_done, 0) != cudaSuccess)
-    rc = rc ? rc : BSA_ERR_CUDA;
-  cleanup();
-  return rc;
+int bsa_forward_fp8_host(const bsa_params* p, const void* hQ, const void* hK, const void* hV,
+                         void* hO, float* hlse, void* dQ, void* dK, void* dV, void* dO,
+                         float* dlse, void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (workspace_bytes < carve(s, nullptr, nullptr) + fp8_carve(s, nullptr, nullptr))
+    return BSA_ERR_INVALID;
+  return forward_host_pipelined(
+      p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, workspace_bytes, stream,
+      [](const bsa_params* sub, void* q, void* k, void* v, void* o, float* l, void* ws,
+         size_t wsb, void* st) { return bsa_forward_fp8(sub, q, k, v, o, l, ws, wsb, st); });
+}
+
+int bsa_forward_threshold_host(const bsa_params* p, float tau, const void* hQ, const void* hK,
+                               const void* hV, void* hO, float* hlse, void* dQ, void* dK,
+                               void* dV, void* dO, float* dlse, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!std::isfinite(tau)) return BSA_ERR_INVALID;
+  if (workspace_bytes <
+      carve(threshold_shape(s), nullptr, nullptr) + bsa::attend_lists_scratch_bytes(s))
+    return BSA_ERR_INVALID;
+  return forward_host_pipelined(
+      p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, workspace_bytes, stream,
+      [tau](const bsa_params* sub, void* q, void* k, void* v, void* o, float* l, void* ws,
+            size_t wsb, void* st) {
+        return bsa_forward_threshold(sub, tau, q, k, v, o, l, ws, wsb, st);
+      });
+}
+
+int bsa_forward_extra_host(const bsa_params* p, int32_t n_extra, const void* hQ, const void* hK,
+                           const void* hV, void* hO, float* hlse, void* dQ, void* dK, void* dV,
+                           void* dO, float* dlse, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!extra_valid(s, n_extra)) return BSA_ERR_INVALID;
+  if (workspace_bytes < carve(s, nullptr, nullptr) + extra_carve(s, n_extra, nullptr, nullptr))
+    return BSA_ERR_INVALID;
+  return forward_host_pipelined(
+      p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, workspace_bytes, stream,
+      [n_extra](const bsa_params* sub, void* q, void* k, void* v, void* o, float* l, void* ws,
+                size_t wsb, void* st) {
+        return bsa_forward_extra(sub, n_extra, q, k, v, o, l, ws, wsb, st);
+      });
+}
+
+int bsa_forward_reblock_host(const bsa_params* p, const void* hQ, const void* hK,
+                             const void* hV, void* hO, float* hlse, void* dQ, void* dK, void* dV,
+                             void* dO, float* dlse, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (workspace_bytes < reblock_forward_carve(s, nullptr, nullptr)) return BSA_ERR_INVALID;
+  return forward_host_pipelined(
+      p, hQ, hK, hV, hO, hlse, dQ, dK, dV, dO, dlse, workspace, workspace_bytes, stream,
+      [](const bsa_params* sub, void* q, void* k, void* v, void* o, float* l, void* ws,
+         size_t wsb, void* st) { return bsa_forward_reblock(sub, q, k, v, o, l, ws, wsb, st); });
 }
 
 const char* bsa_status_string(int status) {

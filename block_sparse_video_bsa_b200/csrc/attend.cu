@@ -16,7 +16,8 @@
 // (top-k lists) both slots have the same tile count.  With variable-length
 // lists (kVar: the count of each row from cnt) each slot runs its own count;
 // the producer and the MMA issuer skip a slot once its tiles are done, and a
-// schedule sorted by count (longest first) pairs rows of similar length.
+// schedule sorted by count inside each head (longest first, heads in order)
+// pairs rows of similar length.
 // 384 threads in three warpgroups; the two softmax warpgroups raise their
 // register budget to 232 and the third lowers its own to 40
 // (128*40 + 256*232 = 384*168, the launch allocation):
@@ -84,9 +85,23 @@ struct Args {
   __nv_bfloat16* O;
   float* lse;
   int* dev_status;
+  // extra tokens (kExtra): ascending token lists [B*H, nb, ecap] and their
+  // counts, the summary rows of partly extra blocks [B*H, nb, scap] (bias,
+  // natural log) and their counts
+  const int32_t* extra;
+  const int32_t* ecnt;
+  const float* side_bias;
+  const int32_t* side_cnt;
+  int ecap, scap;
   int N, nb, pb, nbv, k_eff, kcap, BH;
   int prefix_ctas;    // CTAs that take dense-prefix query-block pairs
   float scale_log2;   // log2(e) / sqrt(128)
+};
+
+// Tensor maps of the extra-token path: K and V as 2-D [B*H*N, 128] with a
+// one-row box (row gathers), the side summary rows as [B*H, nb*scap, 128].
+struct ExtraMaps {
+  CUtensorMap k2, v2, sk, sv;
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx& wc) {
@@ -138,6 +153,17 @@ __device__ __forceinline__ bool listed(const int32_t* row, int lo, int hi, int j
   return false;
 }
 
+// Does the ascending token list row[0..n) hold a token of block j?
+__device__ __forceinline__ bool has_token_of(const int32_t* row, int n, int j) {
+  int lo = 0, hi = n;
+  const int first = j * kBlock;
+  while (lo < hi) {   // first position with token >= first
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(row + mid) < first) lo = mid + 1; else hi = mid;
+  }
+  return lo < n && __ldg(row + lo) < first + kBlock;
+}
+
 // Listed blocks of a video row with a variable-length list, clamped to the
 // row's storage (at least one, so the tile loops and the ragged check stay
 // inside the row).
@@ -146,11 +172,12 @@ __device__ __forceinline__ int list_len(const Args& a, int bh, int qi) {
   return max(1, min(c, min(a.kcap, a.nb)));
 }
 
-template <bool kVar>
+template <bool kVar, bool kExtra>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ks,
-                  const __grid_constant__ CUtensorMap tm_vs, const Args a) {
+                  const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ ExtraMaps em,
+                  const Args a) {
   extern __shared__ __align__(1024) uint8_t sm[];
   Ctl* ctl = reinterpret_cast<Ctl*>(sm + kOffCtl);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -179,12 +206,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     ne1 = list_len(a, pr.bh[1], pr.qi[1]);
   }
   const bool hs0 = video && (ne0 - a.pb < a.nbv), hs1 = video && (ne1 - a.pb < a.nbv);
-  const int T0 = ne0 + (hs0 ? sum_tiles : 0), T1 = ne1 + (hs1 ? sum_tiles : 0);
+  // Extra tokens (video rows only): ec extra tokens in xe gathered tiles after
+  // the listed blocks; sc summary rows of partly extra blocks in st tiles
+  // after the global summary tiles.
+  int ec0 = 0, ec1 = 0, sc0 = 0, sc1 = 0;
+  if (kExtra && video) {
+    ec0 = max(0, min(__ldg(a.ecnt + static_cast<size_t>(pr.bh[0]) * a.nb + pr.qi[0]), a.ecap));
+    ec1 = max(0, min(__ldg(a.ecnt + static_cast<size_t>(pr.bh[1]) * a.nb + pr.qi[1]), a.ecap));
+    sc0 = max(0, min(__ldg(a.side_cnt + static_cast<size_t>(pr.bh[0]) * a.nb + pr.qi[0]), a.scap));
+    sc1 = max(0, min(__ldg(a.side_cnt + static_cast<size_t>(pr.bh[1]) * a.nb + pr.qi[1]), a.scap));
+  }
+  const int xe0 = (ec0 + kBlock - 1) / kBlock, xe1 = (ec1 + kBlock - 1) / kBlock;
+  const int st0 = hs0 ? (sc0 + kBlock - 1) / kBlock : 0, st1 = hs1 ? (sc1 + kBlock - 1) / kBlock : 0;
+  const int T0 = ne0 + xe0 + (hs0 ? sum_tiles : 0) + st0;
+  const int T1 = ne1 + xe1 + (hs1 ? sum_tiles : 0) + st1;
   const int nslots = pr.act1 ? 2 : 1;
   const int steps = (nslots == 2) ? max(T0, T1) : T0;   // tile steps of the CTA
   auto n_exact_of = [&](int s) { return s ? ne1 : ne0; };
   auto tiles_of = [&](int s) { return s ? T1 : T0; };
   auto has_sum_of = [&](int s) { return s ? hs1 : hs0; };
+  auto xe_of = [&](int s) { return s ? xe1 : xe0; };
+  auto ec_of = [&](int s) { return s ? ec1 : ec0; };
+  auto sc_of = [&](int s) { return s ? sc1 : sc0; };
 
   if (tid == 0) {
     for (int i = 0; i < kRing; ++i) {
@@ -217,17 +260,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= 8) {
     reg_dealloc<kControlRegs>();
-    if (warp == kProducerWarp && lane == 0) {
+    if (warp == kProducerWarp && (kExtra || lane == 0)) {
     // ---------------------------------------------------------- producer
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      for (int s = 0; s < nslots; ++s) {
-        mbar_arrive_expect_tx(&ctl->q_full[s], kTileBytes);
-        tma_load_3d(sm + kOffQ + s * kTileBytes, &tm_q, &ctl->q_full[s], 0, pr.qi[s] * kBlock,
-                    pr.bh[s]);
-        tma_load_3d(sm + kOffQ + s * kTileBytes + kSubBytes, &tm_q, &ctl->q_full[s], 64,
-                    pr.qi[s] * kBlock, pr.bh[s]);
+      // With extra tokens the whole warp runs this loop (each lane issues the
+      // row gathers of four rows); otherwise lane 0 alone.  `lead` issues the
+      // tile loads and the barrier operations.
+      const bool lead = lane == 0;
+      auto pwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        if constexpr (kExtra) {
+          bool r = true;
+          if (lead) r = mbar_wait(bar, parity, wc);
+          return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+        } else {
+          return mbar_wait(bar, parity, wc);
+        }
+      };
+      if (lead) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        for (int s = 0; s < nslots; ++s) {
+          mbar_arrive_expect_tx(&ctl->q_full[s], kTileBytes);
+          tma_load_3d(sm + kOffQ + s * kTileBytes, &tm_q, &ctl->q_full[s], 0, pr.qi[s] * kBlock,
+                      pr.bh[s]);
+          tma_load_3d(sm + kOffQ + s * kTileBytes + kSubBytes, &tm_q, &ctl->q_full[s], 64,
+                      pr.qi[s] * kBlock, pr.bh[s]);
+        }
       }
       int seq = 0;
       bool ok = true;
@@ -235,25 +293,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto emit = [&](int s, int t, bool is_v) {
         if (!ok) return;
         const int stage = seq % kRing;
-        if (seq >= kRing && !mbar_wait(&ctl->empty[stage], ((seq / kRing) - 1) & 1, wc)) {
+        if (seq >= kRing && !pwait(&ctl->empty[stage], ((seq / kRing) - 1) & 1)) {
           ok = false;
           return;
         }
-        const CUtensorMap* m;
-        int row;
-        const int n_exact = n_exact_of(s);
-        if (t < n_exact) {
-          row = __ldg(a.idx + (static_cast<size_t>(pr.bh[s]) * a.nb + pr.qi[s]) * a.kcap + t) *
-                kBlock;
-          m = is_v ? &tm_v : &tm_k;
-        } else {
-          row = (u0 + t - n_exact) * kBlock;
-          m = is_v ? &tm_vs : &tm_ks;
-        }
         uint8_t* dst = sm + kOffRing + stage * kTileBytes;
-        mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
-        tma_load_3d(dst, m, &ctl->full[stage], 0, row, pr.bh[s]);
-        tma_load_3d(dst + kSubBytes, m, &ctl->full[stage], 64, row, pr.bh[s]);
+        const int n_exact = n_exact_of(s);
+        if (kExtra && t >= n_exact && t < n_exact + xe_of(s)) {
+          // 128 extra tokens (padded with the first one) gathered row by row:
+          // lane l brings rows 4l..4l+3 of both 64-column halves
+          const int x = t - n_exact, ec = ec_of(s);
+          const int32_t* erow =
+              a.extra + (static_cast<size_t>(pr.bh[s]) * a.nb + pr.qi[s]) * a.ecap;
+          const int first = __ldg(erow);
+          int rr[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int pos = x * kBlock + 4 * lane + k;
+            rr[k] = pr.bh[s] * a.N + (pos < ec ? __ldg(erow + pos) : first);
+          }
+          if (lead) mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
+          __syncwarp();
+          const CUtensorMap* m = is_v ? &em.v2 : &em.k2;
+          tma_gather4(dst + 4 * lane * 128, m, &ctl->full[stage], 0, rr[0], rr[1], rr[2], rr[3]);
+          tma_gather4(dst + kSubBytes + 4 * lane * 128, m, &ctl->full[stage], 64, rr[0], rr[1],
+                      rr[2], rr[3]);
+        } else if (lead) {
+          const CUtensorMap* m;
+          int row, head = pr.bh[s];
+          if (t < n_exact) {
+            row = __ldg(a.idx + (static_cast<size_t>(pr.bh[s]) * a.nb + pr.qi[s]) * a.kcap + t) *
+                  kBlock;
+            m = is_v ? &tm_v : &tm_k;
+          } else {
+            const int v = t - n_exact - xe_of(s);
+            const int gsum = has_sum_of(s) ? sum_tiles : 0;
+            if (!kExtra || v < gsum) {
+              row = (u0 + v) * kBlock;
+              m = is_v ? &tm_vs : &tm_ks;
+            } else {
+              row = pr.qi[s] * a.scap + (v - gsum) * kBlock;
+              m = is_v ? &em.sv : &em.sk;
+            }
+          }
+          mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
+          tma_load_3d(dst, m, &ctl->full[stage], 0, row, head);
+          tma_load_3d(dst + kSubBytes, m, &ctl->full[stage], 64, row, head);
+        }
         ++seq;
       };
       for (int s = 0; s < nslots; ++s) emit(s, 0, false);
@@ -266,9 +352,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: every issued load has landed before the CTA exits (immediate
       // on the normal path, where the MMA warp already waited for them).
-      for (int s = 0; s < nslots; ++s) mbar_wait(&ctl->q_full[s], 0, wc);
-      for (int k = (seq > kRing ? seq - kRing : 0); k < seq; ++k)
-        mbar_wait(&ctl->full[k % kRing], (k / kRing) & 1, wc);
+      if (lead) {
+        for (int s = 0; s < nslots; ++s) mbar_wait(&ctl->q_full[s], 0, wc);
+        for (int k = (seq > kRing ? seq - kRing : 0); k < seq; ++k)
+          mbar_wait(&ctl->full[k % kRing], (k / kRing) & 1, wc);
+      }
     } else if (warp == kMmaWarp && lane == 0) {
     // ---------------------------------------------------------- MMA issuer
       const uint32_t id_s = idesc_bf16_f32(128, 128, 0);
@@ -334,20 +422,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       // in log2 units with -inf where the column is a listed block, a prefix
       // block or past the last block (listed: binary search of the sorted
       // idx row), double buffered against the slot's softmax warps.
+      // With extra tokens, a block that holds some of the row's extra tokens
+      // is masked as well (its remaining tokens come as one of the row's side
+      // summary rows, staged after the global tiles, -inf past their count).
       const int s = warp - 10;
       const int n_exact = n_exact_of(s);
-      const int32_t* idx_row = a.idx + (static_cast<size_t>(pr.bh[s]) * a.nb + pr.qi[s]) * a.kcap;
+      const size_t row_id = static_cast<size_t>(pr.bh[s]) * a.nb + pr.qi[s];
+      const int32_t* idx_row = a.idx + row_id * a.kcap;
       const float* bias_h = a.bias + static_cast<size_t>(pr.bh[s]) * a.nb;
-      for (int v = 0; v < tiles_of(s) - n_exact; ++v) {
+      const int xe = xe_of(s), ec = ec_of(s), sc = sc_of(s);
+      const int gsum = sum_tiles;   // this warp runs only for slots with summaries
+      const int32_t* erow = kExtra ? a.extra + row_id * a.ecap : nullptr;
+      for (int v = 0; v < tiles_of(s) - n_exact - xe; ++v) {
         if (v >= 2 && !warp_wait(&ctl->bias_empty[s][v & 1], ((v >> 1) - 1) & 1, wc)) break;
         float* dst = &ctl->bias_stage[s][v & 1][0];
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           const int c = lane + 32 * q;
-          const int j = (u0 + v) * kBlock + c;
           float b = -INFINITY;
-          if (j >= a.pb && j < a.nb && !listed(idx_row, a.pb, n_exact, j))
-            b = __ldg(bias_h + j) * kLog2e;
+          if (!kExtra || v < gsum) {
+            const int j = (u0 + v) * kBlock + c;
+            if (j >= a.pb && j < a.nb && !listed(idx_row, a.pb, n_exact, j) &&
+                !(kExtra && has_token_of(erow, ec, j)))
+              b = __ldg(bias_h + j) * kLog2e;
+          } else {
+            const int r = (v - gsum) * kBlock + c;
+            if (r < sc) b = __ldg(a.side_bias + row_id * a.scap + r) * kLog2e;
+          }
           dst[c] = b;
         }
         mbar_arrive(&ctl->bias_full[s][v & 1]);
@@ -374,9 +475,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ragged_t = n_exact - 1;
       ragged_cols = a.N - (a.nb - 1) * kBlock;
     }
+    const int xe = xe_of(s);
+    // valid columns of the last extra tile (the token count need not be a
+    // multiple of 128)
+    const int extra_last_t = n_exact + xe - 1;
+    const int extra_last_cols = ec_of(s) - (xe - 1) * kBlock;
     for (int t = 0; ok && t < T; ++t) {
-      const bool exact = t < n_exact;
-      const int v = t - n_exact;   // summary tile index when !exact
+      const bool exact = t < n_exact + xe;
+      const int v = t - n_exact - xe;   // summary tile index when !exact
       if (!warp_wait(&ctl->s_full[s], t & 1, wc)) { ok = false; break; }
       tc_fence_after();
       float x[128];
@@ -395,6 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c >= ragged_cols) x[c] = -INFINITY;
+        }
+        if (kExtra && xe > 0 && t == extra_last_t && extra_last_cols < kBlock) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= extra_last_cols) x[c] = -INFINITY;
         }
       } else {
         if (!warp_wait(&ctl->bias_full[s][v & 1], (v >> 1) & 1, wc)) { ok = false; break; }
@@ -522,13 +633,13 @@ namespace {
 
 // Shared setup of both launches: the kernel's shared-memory attribute (once
 // per device and instantiation) and the arguments common to both.
-template <bool kVar>
+template <bool kVar, bool kExtra = false>
 cudaError_t attend_attr() {
   constexpr size_t smem = kOffCtl + sizeof(Ctl);
   static std::atomic<bool> attr_set[64];
   return once_per_device(attr_set, [] {
-    return cudaFuncSetAttribute(attend_kernel<kVar>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                smem);
+    return cudaFuncSetAttribute(attend_kernel<kVar, kExtra>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
 }
 
@@ -537,6 +648,12 @@ Args attend_args(const Shape& s, const int32_t* idx, const float* bias, void* O,
   a.idx = idx;
   a.cnt = nullptr;
   a.sched = nullptr;
+  a.extra = nullptr;
+  a.ecnt = nullptr;
+  a.side_bias = nullptr;
+  a.side_cnt = nullptr;
+  a.ecap = 0;
+  a.scap = 0;
   a.bias = bias;
   a.O = static_cast<__nv_bfloat16*>(O);
   a.lse = lse;
@@ -554,15 +671,14 @@ Args attend_args(const Shape& s, const int32_t* idx, const float* bias, void* O,
 }
 
 // ---------------------------------------------------------------- schedule
-// Video work items (bh * nbv + qi - pb) ordered by list length, longest
-// first, so that the two slots of a CTA hold rows of similar length and the
-// longest rows start first.  A counting sort: per-CTA shared-memory
-// histograms summed into `bins`, then every CTA scans `bins` from the
-// longest length down, reserves a range per length with one global atomic
-// and scatters its items.  The order inside one length follows the atomics;
-// no row's result depends on the row it is paired with.
+// Video work items (bh * nbv + qi - pb) ordered head by head and, inside a
+// head, by list length, longest first: the two slots of a CTA hold rows of
+// similar length, the longest rows of a head start first, and the K/V of only
+// one or two heads is in flight at a time (the order of the fixed-count path,
+// whose K/V stays in L2).  One CTA per head runs a counting sort of its rows
+// in shared memory; the order inside one length follows the shared-memory
+// atomics, and no row's result depends on the row it is paired with.
 constexpr int kSchedThreads = 512;
-constexpr int kSchedItems = 8192;        // items per CTA
 
 __device__ __forceinline__ int item_len(const int32_t* cnt, int it, int nbv, int nb, int pb,
                                         int kcap) {
@@ -572,36 +688,26 @@ __device__ __forceinline__ int item_len(const int32_t* cnt, int it, int nbv, int
 }
 
 __global__ void __launch_bounds__(kSchedThreads)
-    length_hist_kernel(const int32_t* __restrict__ cnt, int items, int nbv, int nb, int pb,
-                       int kcap, int32_t* __restrict__ bins) {
-  extern __shared__ int h[];             // [nb + 1]
-  for (int b = threadIdx.x; b <= nb; b += kSchedThreads) h[b] = 0;
-  __syncthreads();
-  const int i0 = blockIdx.x * kSchedItems, i1 = min(items, i0 + kSchedItems);
-  for (int it = i0 + threadIdx.x; it < i1; it += kSchedThreads)
-    atomicAdd(&h[item_len(cnt, it, nbv, nb, pb, kcap)], 1);
-  __syncthreads();
-  for (int b = threadIdx.x; b <= nb; b += kSchedThreads)
-    if (h[b]) atomicAdd(&bins[b], h[b]);
-}
-
-__global__ void __launch_bounds__(kSchedThreads)
-    schedule_kernel(const int32_t* __restrict__ cnt, int items, int nbv, int nb, int pb, int kcap,
-                    const int32_t* __restrict__ bins, int32_t* __restrict__ fill,
-                    int32_t* __restrict__ sched) {
+    head_schedule_kernel(const int32_t* __restrict__ cnt, int nbv, int nb, int pb, int kcap,
+                         int32_t* __restrict__ sched) {
   extern __shared__ int sm_sched[];
-  int* start = sm_sched;                 // [nb + 1] items with a longer list
-  int* cur = sm_sched + (nb + 1);        // [nb + 1] local counts, then cursors
+  int* hist = sm_sched;                  // [nb + 1] rows per length
+  int* cur = sm_sched + (nb + 1);        // [nb + 1] first position of each length
   __shared__ int part[kSchedThreads];
   const int tid = threadIdx.x, nbins = nb + 1;
-  // start[b] = sum of bins[b'] over b' > b: thread t scans a contiguous run
-  // of the reversed bins, then the run totals are scanned across the block.
+  const int base = blockIdx.x * nbv;     // this head's items
+  for (int b = tid; b < nbins; b += kSchedThreads) hist[b] = 0;
+  __syncthreads();
+  for (int r = tid; r < nbv; r += kSchedThreads)
+    atomicAdd(&hist[item_len(cnt, base + r, nbv, nb, pb, kcap)], 1);
+  __syncthreads();
+  // cur[b] = rows with a longer list: thread t scans a contiguous run of the
+  // reversed bins, then the run totals are scanned across the block.
   const int per = (nbins + kSchedThreads - 1) / kSchedThreads;
   const int r0 = min(nbins, tid * per), r1 = min(nbins, r0 + per);
   int run = 0;
-  for (int r = r0; r < r1; ++r) run += __ldg(bins + (nb - r));
+  for (int r = r0; r < r1; ++r) run += hist[nb - r];
   part[tid] = run;
-  for (int b = tid; b < nbins; b += kSchedThreads) cur[b] = 0;
   __syncthreads();
   for (int off = 1; off < kSchedThreads; off <<= 1) {      // inclusive scan of part
     const int v = tid >= off ? part[tid - off] : 0;
@@ -611,19 +717,13 @@ __global__ void __launch_bounds__(kSchedThreads)
   }
   int acc = part[tid] - run;                                // exclusive prefix of the run
   for (int r = r0; r < r1; ++r) {
-    start[nb - r] = acc;
-    acc += __ldg(bins + (nb - r));
+    cur[nb - r] = acc;
+    acc += hist[nb - r];
   }
-  const int i0 = blockIdx.x * kSchedItems, i1 = min(items, i0 + kSchedItems);
-  for (int it = i0 + tid; it < i1; it += kSchedThreads)
-    atomicAdd(&cur[item_len(cnt, it, nbv, nb, pb, kcap)], 1);
   __syncthreads();
-  for (int b = tid; b < nbins; b += kSchedThreads)
-    if (cur[b]) cur[b] = start[b] + atomicAdd(&fill[b], cur[b]);
-  __syncthreads();
-  for (int it = i0 + tid; it < i1; it += kSchedThreads) {
-    const int pos = atomicAdd(&cur[item_len(cnt, it, nbv, nb, pb, kcap)], 1);
-    if (pos >= 0 && pos < items) sched[pos] = it;
+  for (int r = tid; r < nbv; r += kSchedThreads) {
+    const int pos = atomicAdd(&cur[item_len(cnt, base + r, nbv, nb, pb, kcap)], 1);
+    if (pos >= 0 && pos < nbv) sched[base + pos] = base + r;
   }
 }
 
@@ -639,15 +739,14 @@ cudaError_t launch_attend(const Shape& s, const AttendMaps& maps, const int32_t*
   if (e != cudaSuccess) return e;
   const Args a = attend_args(s, idx, bias, O, lse);
   const int grid = a.prefix_ctas + (a.BH * s.nbv + 1) / 2;
-  attend_kernel<false><<<grid, kThreads, kOffCtl + sizeof(Ctl), st>>>(maps.q, maps.k, maps.v,
-                                                                      maps.ks, maps.vs, a);
+  const ExtraMaps none{};
+  attend_kernel<false, false><<<grid, kThreads, kOffCtl + sizeof(Ctl), st>>>(
+      maps.q, maps.k, maps.v, maps.ks, maps.vs, none, a);
   return cudaGetLastError();
 }
 
 size_t attend_lists_scratch_bytes(const Shape& s) {
-  const size_t bins = (static_cast<size_t>(s.nb) + 1) * 4;
-  return 2 * ((bins + 255) & ~static_cast<size_t>(255)) +
-         static_cast<size_t>(s.B) * s.H * s.nbv * 4;
+  return static_cast<size_t>(s.B) * s.H * s.nbv * 4;
 }
 
 cudaError_t launch_attend_lists(const Shape& s, const AttendMaps& maps, const int32_t* idx,
@@ -659,31 +758,46 @@ cudaError_t launch_attend_lists(const Shape& s, const AttendMaps& maps, const in
   static std::atomic<bool> sched_attr[64];
   e = once_per_device(sched_attr, [] {
     const int max_dyn = 2 * (16384 + 1) * static_cast<int>(sizeof(int));
-    cudaError_t r = cudaFuncSetAttribute(length_hist_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
-    if (r != cudaSuccess) return r;
-    return cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(head_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 max_dyn);
   });
   if (e != cudaSuccess) return e;
-  const size_t bins_bytes = ((static_cast<size_t>(s.nb) + 1) * 4 + 255) & ~static_cast<size_t>(255);
-  int32_t* bins = static_cast<int32_t*>(scratch);
-  int32_t* fill = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + bins_bytes);
-  int32_t* sched = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + 2 * bins_bytes);
-  const int items = s.B * s.H * s.nbv;
-  if ((e = cudaMemsetAsync(scratch, 0, 2 * bins_bytes, st)) != cudaSuccess) return e;
-  const int sched_grid = (items + kSchedItems - 1) / kSchedItems;
-  length_hist_kernel<<<sched_grid, kSchedThreads, (s.nb + 1) * sizeof(int), st>>>(
-      cnt, items, s.nbv, s.nb, s.pb, kcap, bins);
-  schedule_kernel<<<sched_grid, kSchedThreads, smem_sched, st>>>(cnt, items, s.nbv, s.nb, s.pb,
-                                                                 kcap, bins, fill, sched);
+  int32_t* sched = static_cast<int32_t*>(scratch);
+  head_schedule_kernel<<<s.B * s.H, kSchedThreads, smem_sched, st>>>(cnt, s.nbv, s.nb, s.pb, kcap,
+                                                                     sched);
   Args a = attend_args(s, idx, bias, O, lse);
   a.cnt = cnt;
   a.sched = sched;
   a.kcap = kcap;
   const int grid = a.prefix_ctas + (a.BH * s.nbv + 1) / 2;
-  attend_kernel<true><<<grid, kThreads, kOffCtl + sizeof(Ctl), st>>>(maps.q, maps.k, maps.v,
-                                                                     maps.ks, maps.vs, a);
+  const ExtraMaps none{};
+  attend_kernel<true, false><<<grid, kThreads, kOffCtl + sizeof(Ctl), st>>>(
+      maps.q, maps.k, maps.v, maps.ks, maps.vs, none, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attend_extra(const Shape& s, const AttendMaps& maps,
+                                const AttendExtraMaps& xmaps, const int32_t* idx,
+                                const int32_t* extra, const int32_t* ecnt, int ecap,
+                                const float* bias, const float* side_bias, const int32_t* side_cnt,
+                                int scap, void* O, float* lse, cudaStream_t st) {
+  cudaError_t e = attend_attr<false, true>();
+  if (e != cudaSuccess) return e;
+  Args a = attend_args(s, idx, bias, O, lse);
+  a.extra = extra;
+  a.ecnt = ecnt;
+  a.ecap = ecap;
+  a.side_bias = side_bias;
+  a.side_cnt = side_cnt;
+  a.scap = scap;
+  ExtraMaps em;
+  em.k2 = xmaps.k2;
+  em.v2 = xmaps.v2;
+  em.sk = xmaps.sk;
+  em.sv = xmaps.sv;
+  const int grid = a.prefix_ctas + (a.BH * s.nbv + 1) / 2;
+  attend_kernel<false, true><<<grid, kThreads, kOffCtl + sizeof(Ctl), st>>>(
+      maps.q, maps.k, maps.v, maps.ks, maps.vs, em, a);
   return cudaGetLastError();
 }
 

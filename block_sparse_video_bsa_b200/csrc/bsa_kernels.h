@@ -40,8 +40,13 @@ struct Shape {
 
 cudaError_t launch_pool(const Shape& s, const void* Q, float* qpool, float* anchor,
                         cudaStream_t st);
+// kstat / vstat / lse_blk (optional, all or none): fp32 k~ and v~ (anchor
+// variant) or mean k and mean v (mean variant), [B,H,nb,128], and the block
+// LSE at the anchor (ln n for the mean variant), [B,H,nb].
 cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const float* anchor,
-                             float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st);
+                             float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st,
+                             float* kstat = nullptr, float* vstat = nullptr,
+                             float* lse_blk = nullptr);
 cudaError_t launch_select(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
                           int32_t* cnt, cudaStream_t st);
 // Threshold selection: idx rows of length nb (kcap ignored), cnt per row.
@@ -61,6 +66,17 @@ size_t attend_lists_scratch_bytes(const Shape& s);
 cudaError_t launch_attend_lists(const Shape& s, const AttendMaps& maps, const int32_t* idx,
                                 int kcap, const int32_t* cnt, const float* bias, void* O,
                                 float* lse, void* scratch, cudaStream_t st);
+// Extra tokens: K and V as 2-D [B*H*N, 128] bf16 with a {64, 1} box (row
+// gathers), the side summary rows k~', v~' as [B*H, nb*scap, 128] with the
+// usual {64, 128, 1} box.
+struct AttendExtraMaps {
+  CUtensorMap k2, v2, sk, sv;
+};
+cudaError_t launch_attend_extra(const Shape& s, const AttendMaps& maps,
+                                const AttendExtraMaps& xmaps, const int32_t* idx,
+                                const int32_t* extra, const int32_t* ecnt, int ecap,
+                                const float* bias, const float* side_bias, const int32_t* side_cnt,
+                                int scap, void* O, float* lse, cudaStream_t st);
 // FP8 (e4m3) operands (layouts as bsa_fp8_operands in include/bsa.h).
 struct Fp8Operands {
   void* q8;
@@ -121,6 +137,23 @@ cudaError_t launch_permute_rows(const Shape& s, const void* Q, const void* K, co
                                 cudaStream_t st);
 cudaError_t launch_unpermute_rows(const Shape& s, const void* Op, const float* lsep,
                                   const int32_t* perm, void* O, float* lse, cudaStream_t st);
+
+// Extra tokens (extra.cu).  Candidate-buffer capacity per query block,
+// scratch of the selection, row capacity of the side summary table.
+int extra_cand_cap(int n_extra);
+size_t select_extra_scratch_bytes(const Shape& s, int n_extra);
+int extra_side_cap(const Shape& s, int n_extra);
+// tm_k: K as for the attention ([B*H, N, 128], box {64, 128, 1}, SW128).
+cudaError_t launch_select_extra(const Shape& s, int n_extra, const CUtensorMap& tm_k,
+                                const float* qpool, const int32_t* idx, int kcap,
+                                const int32_t* cnt, int32_t* extra, int32_t* ecnt, void* scratch,
+                                cudaStream_t st);
+cudaError_t launch_extra_summaries(const Shape& s, int n_extra, const void* K, const void* V,
+                                   const float* anchor, const float* kpool, const float* kstat,
+                                   const float* vstat, const float* lse_blk, const int32_t* extra,
+                                   const int32_t* ecnt, void* side_k, void* side_v,
+                                   float* side_bias, int32_t* side_blk, int32_t* side_cnt,
+                                   cudaStream_t st);
 
 cudaError_t launch_expired_wait(int32_t* dev_status, uint64_t timeout_ns, cudaStream_t st);
 

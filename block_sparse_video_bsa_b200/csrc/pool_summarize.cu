@@ -108,7 +108,8 @@ template <int kVariant>  // 0 = anchor-weighted, 1 = mean-pooled
 __global__ void __launch_bounds__(kThreads) summarize_kernel(
     const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
     const float* __restrict__ anchor, float* __restrict__ kpool, __nv_bfloat16* __restrict__ ksum,
-    __nv_bfloat16* __restrict__ vsum, float* __restrict__ bias, int N, int nb, float scale) {
+    __nv_bfloat16* __restrict__ vsum, float* __restrict__ bias, float* __restrict__ kstat,
+    float* __restrict__ vstat, float* __restrict__ lse_blk, int N, int nb, float scale) {
   __shared__ float red[8 * kDim];
   __shared__ float xs[kBlock];
   __shared__ float stat[2];
@@ -217,14 +218,24 @@ __global__ void __launch_bounds__(kThreads) summarize_kernel(
     if (tid < kDim) {
       ksum[o] = __float2bfloat16_rn(kt_d);
       vsum[o] = __float2bfloat16_rn(vt_d);
+      if (kstat) {   // fp32 statistics for the summaries of partial blocks
+        kstat[o] = kt_d;
+        vstat[o] = vt_d;
+      }
     }
     if (tid == 0) bias[bh * nb + blk] = lse - ((red[0] + red[1]) + (red[2] + red[3])) * scale;
+    if (tid == 0 && lse_blk) lse_blk[bh * nb + blk] = lse;
   } else {
     if (tid < kDim) {
       ksum[o] = __float2bfloat16_rn(ksum_d * inv_n);
       vsum[o] = __float2bfloat16_rn(vt_d * inv_n);
+      if (kstat) {
+        kstat[o] = ksum_d * inv_n;
+        vstat[o] = vt_d * inv_n;
+      }
     }
     if (tid == 0) bias[bh * nb + blk] = logf(static_cast<float>(n));
+    if (tid == 0 && lse_blk) lse_blk[bh * nb + blk] = logf(static_cast<float>(n));
   }
 }
 
@@ -240,7 +251,8 @@ cudaError_t launch_pool(const Shape& s, const void* Q, float* qpool, float* anch
 }
 
 cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const float* anchor,
-                             float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st) {
+                             float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st,
+                             float* kstat, float* vstat, float* lse_blk) {
   const dim3 grid(s.nb, s.B * s.H);
   const float scale = 0.088388347648318440550f;  // 1 / sqrt(128)
   auto Kp = static_cast<const __nv_bfloat16*>(K);
@@ -248,11 +260,11 @@ cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const
   auto ks = static_cast<__nv_bfloat16*>(ksum);
   auto vs = static_cast<__nv_bfloat16*>(vsum);
   if (s.variant == 0)
-    summarize_kernel<0><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias, s.N, s.nb,
-                                                   scale);
+    summarize_kernel<0><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias, kstat,
+                                                   vstat, lse_blk, s.N, s.nb, scale);
   else
-    summarize_kernel<1><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias, s.N, s.nb,
-                                                   scale);
+    summarize_kernel<1><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias, kstat,
+                                                   vstat, lse_blk, s.N, s.nb, scale);
   return cudaGetLastError();
 }
 

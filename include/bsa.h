@@ -159,6 +159,30 @@ int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK,
                      void* dV, void* dO, float* dlse, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/* The same host-buffer pipeline for the options: the FP8 forward
+ * (bsa_forward_fp8, workspace bsa_forward_fp8_workspace_bytes), threshold
+ * selection (bsa_forward_threshold, workspace
+ * bsa_forward_threshold_workspace_bytes), extra tokens (bsa_forward_extra,
+ * workspace bsa_forward_extra_workspace_bytes) and adaptive reblocking
+ * (bsa_forward_reblock, workspace bsa_forward_reblock_workspace_bytes), each
+ * chunk's forward being the option's own forward on a sub-call of its
+ * slices.  Arguments, streams and error behaviour as bsa_forward_host. */
+int bsa_forward_fp8_host(const bsa_params* p, const void* hQ, const void* hK, const void* hV,
+                         void* hO, float* hlse, void* dQ, void* dK, void* dV, void* dO,
+                         float* dlse, void* workspace, size_t workspace_bytes, void* stream);
+int bsa_forward_threshold_host(const bsa_params* p, float tau, const void* hQ, const void* hK,
+                               const void* hV, void* hO, float* hlse, void* dQ, void* dK,
+                               void* dV, void* dO, float* dlse, void* workspace,
+                               size_t workspace_bytes, void* stream);
+int bsa_forward_extra_host(const bsa_params* p, int32_t n_extra, const void* hQ, const void* hK,
+                           const void* hV, void* hO, float* hlse, void* dQ, void* dK, void* dV,
+                           void* dO, float* dlse, void* workspace, size_t workspace_bytes,
+                           void* stream);
+int bsa_forward_reblock_host(const bsa_params* p, const void* hQ, const void* hK,
+                             const void* hV, void* hO, float* hlse, void* dQ, void* dK, void* dV,
+                             void* dO, float* dlse, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
 /* ---- forward without any allocation ---------------------------------- */
 
 /* Size of the static device scratch behind bsa_forward_noalloc: 64 MiB. */
@@ -358,6 +382,101 @@ size_t bsa_forward_threshold_workspace_bytes(const bsa_params* p);
 int bsa_forward_threshold(const bsa_params* p, float tau, const void* Q, const void* K,
                           const void* V, void* O, float* lse, void* workspace,
                           size_t workspace_bytes, void* stream);
+
+/* ---- option: extra top-scoring tokens per query block -------------------
+ * "H3 Sparse Attention" (comfy.icu, WAS node page), "The inputs that
+ * matter": besides its chosen blocks, each query block reads a number of
+ * individually chosen top-scoring tokens (`extra_tokens`, 256 by default, 0
+ * the fastest setting).  This library's readings (the page gives no
+ * formula):
+ *   - token u scores s_iu = qhat_i . k_u / sqrt(D) for query block i (the
+ *     token analogue of the pooled block score);
+ *   - the candidates are the video tokens of the video blocks NOT listed for
+ *     i; dense-prefix query blocks take none;
+ *   - the min(n_extra, #candidates) highest scores are taken, ties to the
+ *     lower token index;
+ *   - every key token enters the softmax once: an extra token is read
+ *     exactly, so the summary row of its block stands for the block's
+ *     remaining tokens (the block-summary definition of bsa_summarize over
+ *     those tokens only; no row once all of the block's tokens are extra).
+ * The selection computes the scores on the tensor cores with qhat split into
+ * bf16 hi + lo parts (about 16 significant bits, K is exact bf16) and fp32
+ * accumulation, so two tokens whose scores differ by less than about
+ * 2^-16 * sum_d |qhat_d k_ud| / sqrt(D) may be ordered either way.
+ * 0 <= n_extra <= BSA_MAX_EXTRA_TOKENS, and B*H*N < 2^31, else
+ * BSA_ERR_INVALID.  These calls use the fixed top-k lists of bsa_select. */
+#define BSA_MAX_EXTRA_TOKENS 512
+
+/* Row capacity scap of the side summary table: min(n_extra, nbv) rounded up
+ * to a multiple of 128 (0 for n_extra = 0); -1 for invalid arguments. */
+int32_t bsa_extra_side_capacity(const bsa_params* p, int32_t n_extra);
+
+/* bsa_summarize plus the fp32 statistics the side summaries start from:
+ * kstat, vstat fp32 [B,H,nb,D] = k~ and v~ before bf16 rounding (anchor
+ * variant) or the mean key and mean value (mean variant); lse_blk fp32
+ * [B,H,nb] = the block's log-sum-exp at the anchor, LSE_j (ln n_j for the
+ * mean variant).  Same reads as bsa_summarize (K and V once). */
+int bsa_summarize_stats(const bsa_params* p, const void* K, const void* V, const float* anchor,
+                        float* kpool, void* ksum, void* vsum, float* bias, float* kstat,
+                        float* vstat, float* lse_blk, void* stream);
+
+/* Scratch of bsa_select_extra: one candidate buffer per video query block
+ * (0 for n_extra = 0); 0 also for invalid arguments. */
+size_t bsa_select_extra_workspace_bytes(const bsa_params* p, int32_t n_extra);
+
+/* Extra tokens of every query block.  qpool as bsa_pool wrote it, K bf16
+ * [B,H,N,D], idx/cnt as bsa_select wrote them.  Writes extra int32
+ * [B,H,nb,n_extra] (token indices within the head, ascending, -1 padded) and
+ * ecnt int32 [B,H,nb] (0 for dense-prefix query blocks).  `workspace`
+ * (device, 256-byte aligned, bsa_select_extra_workspace_bytes bytes; may be
+ * NULL for n_extra = 0) holds the candidate buffers; its contents need not be
+ * initialised.  Deterministic. */
+int bsa_select_extra(const bsa_params* p, int32_t n_extra, const float* qpool, const void* K,
+                     const int32_t* idx, const int32_t* cnt, int32_t* extra, int32_t* ecnt,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Summary rows of the blocks that lose some (not all) of their tokens to a
+ * query block's extra tokens.  For video query block i, its affected blocks
+ * j in ascending order get row a of
+ *   side_k, side_v bf16 [B,H,nb,scap,D]  (k~', v~' over the remaining tokens),
+ *   side_bias fp32 [B,H,nb,scap]         (bias', natural log; anchor variant:
+ *                                          LSE'_j - anchor . bf16(k~')/sqrt(D),
+ *                                          mean variant: ln(remaining count)),
+ *   side_blk int32 [B,H,nb,scap]         (j),
+ * side_cnt int32 [B,H,nb] = number of rows (0 for prefix query blocks).  Rows
+ * from side_cnt up to the next multiple of 128 are zero with bias -inf and
+ * block -1.  Anchor variant: the rows are downdates of kstat/vstat/lse_blk by
+ * the extra tokens' softmax weights at the anchor, recomputed from the
+ * remaining rows when less than 2^-6 of the block's anchor mass remains;
+ * mean variant: downdates of the mean key (kpool) and mean value (vstat). */
+int bsa_extra_summaries(const bsa_params* p, int32_t n_extra, const void* K, const void* V,
+                        const float* anchor, const float* kpool, const float* kstat,
+                        const float* vstat, const float* lse_blk, const int32_t* extra,
+                        const int32_t* ecnt, void* side_k, void* side_v, float* side_bias,
+                        int32_t* side_blk, int32_t* side_cnt, void* stream);
+
+/* Step 6 with extra tokens: as bsa_attend, plus for every video query row
+ * the extra tokens of its block as exact logits (rows gathered from K and V
+ * by index), and in the compressed branch the global summary rows of blocks
+ * that hold any of the row's extra tokens replaced by the row's side summary
+ * rows.  With n_extra = 0 (ecnt and side_cnt all zero) it computes exactly
+ * what bsa_attend computes. */
+int bsa_attend_extra(const bsa_params* p, int32_t n_extra, const void* Q, const void* K,
+                     const void* V, const int32_t* idx, const int32_t* cnt, const int32_t* extra,
+                     const int32_t* ecnt, const void* ksum, const void* vsum, const float* bias,
+                     const void* side_k, const void* side_v, const float* side_bias,
+                     const int32_t* side_cnt, void* O, float* lse, void* stream);
+
+/* Workspace of bsa_forward_extra: bsa_workspace_bytes(p) followed by the
+ * statistics, lists, side table and candidate buffers (0 if invalid). */
+size_t bsa_forward_extra_workspace_bytes(const bsa_params* p, int32_t n_extra);
+
+/* bsa_pool, bsa_summarize_stats, bsa_select, bsa_select_extra,
+ * bsa_extra_summaries, bsa_attend_extra in order on `stream`, intermediates in
+ * the caller's workspace (256-byte aligned). */
+int bsa_forward_extra(const bsa_params* p, int32_t n_extra, const void* Q, const void* K,
+                      const void* V, void* O, float* lse, void* workspace, size_t workspace_bytes,
+                      void* stream);
 
 /* Human-readable name of a bsa_status value (static string). */
 const char* bsa_status_string(int status);

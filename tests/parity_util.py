@@ -244,3 +244,159 @@ def check_head_threshold(buf, Q, K, V, b, h, tau, prefix, variant, check_lse=Tru
         check_lse_bound(host(buf["lse"][b, h]), Qh, ref, lse_ref, pb, variant, N)
     kept = np.array([len(l) - pb for l in lists[pb:]])
     return m, r, differ, kept
+
+
+# ------------------------------------------------------------ extra tokens
+
+# Ordering slack of the token scores the GPU ranks: qhat enters the tensor
+# cores as bf16 hi + lo (each component within 2^-18 of qhat) and the 256
+# products of a score accumulate in fp32, so a GPU score is within
+# (2^-18 + 2^-16) * sum_d |qhat_d k_ud| of the exact dot product; divided by
+# sqrt(d) on the oracle's scale.  2^-15 covers both terms.
+EXTRA_GAP_REL = 2.0 ** -15
+
+
+def run_stages_extra(Q, K, V, top_k, n_extra, prefix, variant, with_lse=True):
+    """The extra-token path stage by stage through its C entry points."""
+    B, H, N, _ = Q.shape
+    p = bsa.params(B, H, N, top_k, prefix, variant)
+    buf = bsa.stage_buffers(B, H, N, top_k, prefix, variant, device=Q.device)
+    buf.update(bsa.extra_buffers(B, H, N, top_k, n_extra, prefix, variant, device=Q.device))
+    bsa.bsa_pool(p, Q, buf["qpool"], buf["anchor"])
+    bsa.bsa_summarize_stats(p, K, V, buf["anchor"], buf["kpool"], buf["ksum"], buf["vsum"],
+                            buf["bias"], buf["kstat"], buf["vstat"], buf["lse_blk"])
+    bsa.bsa_select(p, buf["qpool"], buf["kpool"], buf["idx"], buf["cnt"])
+    bsa.bsa_select_extra(p, n_extra, buf["qpool"], K, buf["idx"], buf["cnt"], buf["extra"],
+                         buf["ecnt"], buf["cand"])
+    bsa.bsa_extra_summaries(p, n_extra, K, V, buf["anchor"], buf["kpool"], buf["kstat"],
+                            buf["vstat"], buf["lse_blk"], buf["extra"], buf["ecnt"], buf["side_k"],
+                            buf["side_v"], buf["side_bias"], buf["side_blk"], buf["side_cnt"])
+    O = torch.empty_like(Q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=Q.device) if with_lse else None
+    bsa.bsa_attend_extra(p, n_extra, Q, K, V, buf["idx"], buf["cnt"], buf["extra"], buf["ecnt"],
+                         buf["ksum"], buf["vsum"], buf["bias"], buf["side_k"], buf["side_v"],
+                         buf["side_bias"], buf["side_cnt"], O, lse)
+    torch.cuda.synchronize()
+    buf["O"] = O
+    buf["lse"] = lse
+    return buf
+
+
+def check_extra_selection(extra_rows, ecnt_row, s, lists, Kh, qpool, n_extra, pb, N):
+    """GPU extra tokens of one head vs the oracle's choice over the same block
+    lists: valid candidates, the right count, and the same set except tokens
+    whose oracle scores lie within the derived ordering slack of the row's
+    n-th score.  Returns the GPU's extra lists."""
+    from oracle import bsa_oracle_extra as ox
+    want = ox.select_extra_tokens(s, lists, pb, n_extra, N)
+    bounds = orc.block_bounds(N)
+    nb = len(bounds)
+    absk = np.abs(Kh)
+    got_all = []
+    for i in range(nb):
+        c = int(ecnt_row[i])
+        got = [int(u) for u in extra_rows[i, :c]] if n_extra > 0 else []
+        if n_extra > 0:
+            assert all(int(u) == -1 for u in extra_rows[i, c:]), f"padding of row {i}"
+        got_all.append(np.array(got, dtype=np.int64))
+        w = [int(u) for u in want[i]]
+        assert c == len(w), (i, c, len(w))
+        if got == w:
+            continue
+        assert i >= pb, f"prefix row {i}"
+        listed = set(int(j) for j in lists[i])
+        assert got == sorted(set(got)), f"row {i} not ascending / unique"
+        assert all(u >= pb * 128 and (u // 128) not in listed and u < N for u in got), i
+        cand = np.concatenate([np.arange(*bounds[j]) for j in range(pb, nb) if j not in listed])
+        nth = np.sort(s[i, cand])[::-1][len(w) - 1]
+        for u in set(got) ^ set(w):
+            gap = EXTRA_GAP_REL * float(np.abs(qpool[i]) @ absk[u]) / np.sqrt(Kh.shape[1]) + 1e-7
+            assert abs(s[i, u] - nth) <= gap, (i, u, s[i, u], nth, gap)
+    return got_all
+
+
+def check_side_rows(buf, b, h, Kh, Vh, anchor, lists, extras, variant, pb, N):
+    """The GPU's summary rows of partly extra blocks against the summary
+    definition over the remaining tokens (the oracle's summary_of_tokens)."""
+    from oracle import bsa_oracle_extra as ox
+    bounds = orc.block_bounds(N)
+    nb = len(bounds)
+    sk, sv = host(buf["side_k"][b, h]), host(buf["side_v"][b, h])
+    sb, sj, sc = host(buf["side_bias"][b, h]), host(buf["side_blk"][b, h]), host(buf["side_cnt"][b, h])
+    d = Kh.shape[1]
+    for i in range(nb):
+        if i < pb:
+            assert int(sc[i]) == 0
+            continue
+        ex = set(int(u) for u in extras[i])
+        listed = set(int(j) for j in lists[i])
+        rows = []
+        for j in range(pb, nb):
+            if j in listed:
+                continue
+            toks = np.arange(*bounds[j])
+            rest = np.array([t for t in toks if t not in ex], dtype=np.int64)
+            if 0 < len(rest) < len(toks):
+                rows.append((j, ox.summary_of_tokens(Kh, Vh, rest, anchor, variant)))
+        assert int(sc[i]) == len(rows), (i, int(sc[i]), len(rows))
+        for a_, (j, (k_, v_, b_)) in enumerate(rows):
+            assert int(sj[i, a_]) == j, (i, a_, int(sj[i, a_]), j)
+            np.testing.assert_allclose(sk[i, a_], k_, rtol=SUM_RTOL, atol=SUM_ATOL)
+            np.testing.assert_allclose(sv[i, a_], v_, rtol=SUM_RTOL, atol=SUM_ATOL)
+            tol = (BF16_U * float(np.abs(k_) @ np.abs(anchor)) / np.sqrt(d) if variant == "anchor"
+                   else 0.0) + FP32_SLACK
+            assert abs(float(sb[i, a_]) - b_) <= tol, (i, j, float(sb[i, a_]), b_, tol)
+        pad = -(-len(rows) // 128) * 128
+        if pad > len(rows):
+            assert np.all(sk[i, len(rows):pad] == 0) and np.all(np.isneginf(sb[i, len(rows):pad]))
+
+
+def check_head_extra(buf, Q, K, V, b, h, top_k, n_extra, prefix, variant, check_lse=True,
+                     query_blocks=None):
+    """Per-stage parity of one (b, h) slice of the extra-token path: stages,
+    lists, fp32 block statistics, the extra tokens, the side summary rows, then
+    O and lse against the oracle's attention over the GPU's (validated) lists
+    and extra tokens on every row (or on ``query_blocks``)."""
+    from oracle import bsa_oracle_extra as ox
+    N = Q.shape[2]
+    Qh, Kh, Vh = host(Q[b, h]), host(K[b, h]), host(V[b, h])
+    ref = ox.forward_head_extra(Qh, Kh, Vh, top_k, 0, prefix, variant, query_blocks=set())
+    ref["scores"] = orc.block_scores(ref["qpool"], ref["kpool"])
+    pb = prefix // 128
+    check_stages(buf, ref, b, h, pb)
+    idx_rows, cnt_row = host(buf["idx"][b, h]), host(buf["cnt"][b, h])
+    check_selection(idx_rows, cnt_row, ref, pb, top_k)
+    lists = gpu_lists(idx_rows, cnt_row)
+    # fp32 block statistics (the GPU's own fp32 sums; oracle fp64)
+    d = Kh.shape[1]
+    v = slice(pb, None)
+    np.testing.assert_allclose(host(buf["kstat"][b, h])[v], ref["ksum"][v], rtol=1e-5, atol=1e-5)
+    np.testing.assert_allclose(host(buf["vstat"][b, h])[v], ref["vsum"][v], rtol=1e-5, atol=1e-5)
+    if variant == "anchor":
+        lse_ref = ref["bias"] + ref["ksum"] @ ref["anchor"] / np.sqrt(d)
+    else:
+        lse_ref = np.log([hi - lo for lo, hi in orc.block_bounds(N)])
+    np.testing.assert_allclose(host(buf["lse_blk"][b, h])[v], lse_ref[v], rtol=1e-5, atol=1e-5)
+    s = ox.token_scores(ref["qpool"], Kh)
+    extras = check_extra_selection(host(buf["extra"][b, h]), host(buf["ecnt"][b, h]), s, lists,
+                                   Kh, ref["qpool"], n_extra, pb, N)
+    check_side_rows(buf, b, h, Kh, Vh, ref["anchor"], lists, extras, variant, pb, N)
+    O_ref, lse_r = ox.attend_extra(Qh, Kh, Vh, lists, extras, ref["ksum"], ref["vsum"],
+                                   ref["bias"], ref["anchor"], variant, pb,
+                                   query_blocks=query_blocks)
+    O_gpu = host(buf["O"][b, h])
+    rows = np.arange(N) if query_blocks is None else rows_of_blocks(N, query_blocks)
+    m, r = check_output(O_gpu[rows], O_ref[rows], len(rows))
+    if check_lse and buf.get("lse") is not None:
+        # every summary logit (global or side row) moves by at most
+        # 2^-8 * sum_d |q_d - c_d| |k~_d| / sqrt(d) through the bf16 rounding
+        # of the summary key the MMA reads
+        centre = ref["anchor"][None, :] if variant == "anchor" else 0.0
+        sk_all, scnt = host(buf["side_k"][b, h]), host(buf["side_cnt"][b, h])
+        side_rows = [sk_all[i, :int(scnt[i])] for i in range(len(scnt)) if int(scnt[i]) > 0]
+        kall = np.abs(np.concatenate([ref["ksum"][pb:]] + side_rows, axis=0))
+        qd = np.abs(Qh[rows] - centre)
+        tol = BF16_U * (qd @ kall.T).max(axis=1) / np.sqrt(d) + FP32_SLACK
+        err = np.abs(host(buf["lse"][b, h])[rows] - lse_r[rows])
+        assert (err <= tol).all(), f"lse err {err.max()} (bound {tol.min()})"
+    return m, r, extras

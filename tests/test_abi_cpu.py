@@ -181,15 +181,15 @@ def test_reblock_scratch_follows_the_tree_shape(B, H, N, prefix):
 
 def test_threshold_sizes():
     # lists of up to nb blocks; the schedule holds one int per video query
-    # block plus two length histograms
+    # block
     p = _p()
     bh, nb = 56, 295
     assert bsa.bsa_threshold_capacity(p) == nb
     assert bsa.bsa_threshold_capacity(_p(top_k=0)) == -1
     r256 = lambda x: (x + 255) // 256 * 256
-    assert bsa.bsa_attend_lists_workspace_bytes(p) == 2 * r256((nb + 1) * 4) + bh * nb * 4
+    assert bsa.bsa_attend_lists_workspace_bytes(p) == bh * nb * 4
     pp = _p(N=103_996, prefix=512)
-    assert bsa.bsa_attend_lists_workspace_bytes(pp) == 2 * r256((813 + 1) * 4) + bh * 809 * 4
+    assert bsa.bsa_attend_lists_workspace_bytes(pp) == bh * 809 * 4
     fw = bsa.bsa_forward_threshold_workspace_bytes(p)
     fixed = bsa.bsa_workspace_bytes(p)             # idx rows of 64 there, of 295 here
     assert fw - bsa.bsa_attend_lists_workspace_bytes(p) - fixed == \
@@ -220,3 +220,57 @@ def test_threshold_arguments_rejected_before_launch():
     assert L.bsa_attend_lists(ctypes.byref(pp), a, a, a, a, 812, a, a, a, a, a, None, a, big,
                               None) == bsa.BSA_ERR_INVALID
     assert L.bsa_forward_threshold(P, 1.0, a, a, a, a, None, a, 16, None) == bsa.BSA_ERR_INVALID
+
+
+def test_extra_token_sizes():
+    # side rows: min(n_extra, nbv) rounded up to 128; candidate buffers of 768
+    # keys per video query block up to 256 extra tokens, 1280 above
+    p = _p()
+    bh, nb = 56, 295
+    assert bsa.bsa_extra_side_capacity(p, 256) == 256
+    assert bsa.bsa_extra_side_capacity(p, 100) == 128
+    assert bsa.bsa_extra_side_capacity(p, 0) == 0
+    assert bsa.bsa_extra_side_capacity(bsa.params(1, 1, 1000, 3), 300) == 128   # nbv = 8
+    assert bsa.bsa_extra_side_capacity(p, 513) == -1 and bsa.bsa_extra_side_capacity(p, -1) == -1
+    assert bsa.bsa_select_extra_workspace_bytes(p, 256) == bh * nb * 768 * 8
+    assert bsa.bsa_select_extra_workspace_bytes(p, 257) == bh * nb * 1280 * 8
+    assert bsa.bsa_select_extra_workspace_bytes(p, 0) == 0
+    r256 = lambda x: (x + 255) // 256 * 256
+    blocks = bh * nb
+    want = sum(r256(x) for x in (blocks * 512, blocks * 512, blocks * 4, blocks * 256 * 4,
+                                 blocks * 4, blocks * 256 * 256, blocks * 256 * 256,
+                                 blocks * 256 * 4, blocks * 256 * 4, blocks * 4,
+                                 blocks * 768 * 8))
+    assert bsa.bsa_forward_extra_workspace_bytes(p, 256) == bsa.bsa_workspace_bytes(p) + want
+    # the row gathers use 32-bit row coordinates
+    assert bsa.bsa_forward_extra_workspace_bytes(bsa.params(64, 16, 1 << 21, 64), 256) == 0
+
+
+def test_extra_token_arguments_rejected_before_launch():
+    L = bsa.lib()
+    p = _p()
+    P = ctypes.byref(p)
+    a = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    big = 1 << 40
+    for n in (-1, 513):
+        assert L.bsa_select_extra(P, n, a, a, a, a, a, a, a, big, None) == bsa.BSA_ERR_INVALID
+        assert L.bsa_forward_extra(P, n, a, a, a, a, None, a, big, None) == bsa.BSA_ERR_INVALID
+        assert L.bsa_attend_extra(P, n, *([a] * 14), a, None, None) == bsa.BSA_ERR_INVALID
+        assert L.bsa_extra_summaries(P, n, *([a] * 14), None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_select_extra(P, 256, a, a, a, a, a, a, a, 16, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_select_extra(P, 256, a, a, a, a, None, a, a, big, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_select_extra(P, 256, odd, a, a, a, a, a, a, big, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_select_extra(P, 256, a, a, a, a, a, a, odd, big, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_forward_extra(P, 256, a, a, a, a, None, a, 16, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_forward_extra(P, 256, a, a, a, odd, None, a, big, None) == bsa.BSA_ERR_ALIGN
+    # the anchor variant needs the anchor; the side table needs 16-byte rows
+    args = [a] * 14
+    args[2] = None
+    assert L.bsa_extra_summaries(P, 256, *args, None) == bsa.BSA_ERR_INVALID
+    args = [a] * 14
+    args[9] = odd
+    assert L.bsa_extra_summaries(P, 256, *args, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_attend_extra(P, 256, *([a] * 14), odd, None, None) == bsa.BSA_ERR_ALIGN
+    assert L.bsa_summarize_stats(P, a, a, a, a, a, a, a, None, a, a, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_summarize_stats(P, a, a, a, a, a, a, a, odd, a, a, None) == bsa.BSA_ERR_ALIGN

@@ -122,3 +122,50 @@ def test_parallelism_labels_name_the_split():
     assert "all-gathered" in bench.parallelism_label(A, 8, 56, 7, True)
     A.shard = None
     assert "B=8 x 56 heads" in bench.parallelism_label(A, 8, 448, 56, False)
+
+
+def test_effective_pairs_with_extra_tokens_match_the_oracle_count():
+    # the device arrays (lists, extra tokens, side-row counts) give the same
+    # computed-pair count as the oracle's head with its extra tokens
+    from oracle import bsa_oracle_extra as ox
+    r = np.random.default_rng(1)
+    N, d, P, n_extra = 1500, 16, 256, 100
+    Q, K, V = (r.standard_normal((N, d)) for _ in range(3))
+    out = ox.forward_head_extra(Q, K, V, 3, n_extra, P, query_blocks=set())
+    nb = len(out["lists"])
+    idx = np.full((1, nb, nb), -1, dtype=np.int64)
+    cnt = np.zeros((1, nb), dtype=np.int64)
+    extra = np.full((1, nb, n_extra), -1, dtype=np.int64)
+    ecnt = np.zeros((1, nb), dtype=np.int64)
+    side = np.zeros((1, nb), dtype=np.int64)
+    bounds = orc.block_bounds(N)
+    for i, L in enumerate(out["lists"]):
+        idx[0, i, :len(L)] = L
+        cnt[0, i] = len(L)
+        e = out["extras"][i]
+        extra[0, i, :len(e)] = e
+        ecnt[0, i] = len(e)
+        blocks = set(int(u) // 128 for u in e)
+        side[0, i] = sum(1 for j in blocks
+                         if sum(1 for u in e if int(u) // 128 == j) < bounds[j][1] - bounds[j][0])
+    assert ecnt[0, P // 128:].min() == n_extra
+    assert bench.effective_pairs_extra(idx, cnt, extra, ecnt, side, N, P) == \
+        bench.oracle_pairs(N, out, P // 128)
+    # no extra tokens: the top-k count
+    assert bench.effective_pairs_extra(idx, cnt, extra, ecnt * 0, side * 0, N, P) == \
+        bench.effective_pairs(idx, cnt, N, P)
+
+
+def test_extra_token_options():
+    for bad in (["--extra-tokens", "256", "--tau", "1.0"], ["--extra-tokens", "600"],
+                ["--extra-tokens", "256", "--precision", "fp8"]):
+        out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *bad],
+                             capture_output=True, text=True, timeout=120, cwd=ROOT)
+        assert out.returncode != 0 and "--extra-tokens" in out.stderr
+    out = subprocess.run(
+        [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+         "tiny_iid", "--extra-tokens", "128", "--steps", "1", "--warmup", "0"],
+        capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    line = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
+    assert line["config"]["extra_tokens"] == 128 and line["value"] > 0
