@@ -16,15 +16,17 @@
 //                        split into bf16 hi + lo (qhat ~= hi + lo to ~16 bits;
 //                        K is exact bf16), B = one 128-token key block from
 //                        a 4-stage TMA ring, D = 128 x 128 fp32 in TMEM
-//                        (double buffered).  One thread per query block keeps
+//                        (four buffers).  One thread per query block keeps
 //                        a running threshold and appends the candidates above
 //                        it to its own buffer in global memory as 64-bit keys
 //                        (order-preserving score bits << 32 | ~token, so a
 //                        larger key is a higher score, then a lower index);
 //                        when a buffer fills, the warp compacts it to the
-//                        n_extra largest keys by an 8-bit radix select and
-//                        raises the threshold to the smallest kept key.  The
-//                        kept tokens are written in ascending order.
+//                        n_extra largest keys (bitwise binary search with
+//                        warp-wide counts) and raises the threshold to the
+//                        smallest kept key.
+//  extra_finish_kernel   one warp per query block: the n_extra largest keys
+//                        of its buffer, written as tokens in ascending order.
 //  extra_summary_kernel  one CTA per video query block: the extra tokens form
 //                        runs by block (the list is ascending); for each
 //                        block that keeps some tokens, its summary over the
@@ -53,16 +55,16 @@ constexpr uint32_t kOffAhi = 0;
 constexpr uint32_t kOffAlo = kTileB;
 constexpr uint32_t kOffRingB = 2 * kTileB;
 constexpr uint32_t kOffSelCtl = kOffRingB + kSelRing * kTileB;
-constexpr uint32_t kSelTmemCols = 256;
+constexpr uint32_t kSelTmemCols = 512;
+constexpr int kDBuf = 4;   // score buffers in TMEM (the selection warps may drift apart)
 
 struct SelCtl {
   uint64_t full[kSelRing], empty[kSelRing];
-  uint64_t d_full[2], d_empty[2];
+  uint64_t d_full[kDBuf], d_empty[kDBuf];
   uint64_t fin;
   uint32_t tmem_base;
   int abort_flag;
   int skip;
-  uint32_t scratch[4][512];   // per selection warp: radix histogram / sort buffer
 };
 static_assert(kOffSelCtl + sizeof(SelCtl) <= 227 * 1024, "shared memory budget");
 
@@ -71,6 +73,8 @@ struct SelArgs {
   const int32_t* idx;          // [BH, nb, kcap]
   const int32_t* cnt;          // [BH, nb]
   unsigned long long* cand;    // [BH * nbv, kCap] candidate buffers
+  int32_t* bcnt;               // [BH * nbv] keys left in each buffer
+  int rows_v;                  // BH * nbv
   int32_t* extra;              // [BH, nb, n_extra]
   int32_t* ecnt;               // [BH, nb]
   int* dev_status;
@@ -95,80 +99,88 @@ __device__ __forceinline__ float key_score(unsigned long long key) {
 
 // Warp-cooperative: the `target` largest of the `count` keys in buf[0..count)
 // (all distinct, non-zero), left in buf[0..target) in any order.  Returns the
-// smallest kept key.  8-bit radix select over the 64-bit keys, histograms in
-// the warp's shared scratch.  Requires target <= count <= 32 * kSlots.
+// smallest kept key.  The target-th largest key is found by a bitwise binary
+// search with warp-wide counts (no shared-memory atomics): first on the score
+// half of the keys, then, when several keys share that score, on the token
+// half among them (a single one is found by a minimum).  Requires
+// 1 <= target <= count <= 32 * kSlots.
 template <int kSlots>
-__device__ unsigned long long compact_keys(unsigned long long* buf, int count, int target,
-                                           uint32_t* hist) {
+__device__ unsigned long long compact_keys(unsigned long long* buf, int count, int target) {
   const int lane = threadIdx.x & 31;
   __syncwarp();   // the owner's appends are visible to every lane
-  unsigned long long e[kSlots];
+  uint32_t hi[kSlots], lo[kSlots];
 #pragma unroll
   for (int k = 0; k < kSlots; ++k) {
     const int p = lane + 32 * k;
-    e[k] = p < count ? buf[p] : 0ull;
+    const unsigned long long e = p < count ? buf[p] : 0ull;
+    hi[k] = static_cast<uint32_t>(e >> 32);
+    lo[k] = static_cast<uint32_t>(e);
   }
   __syncwarp();
-  unsigned long long prefix = 0, pmask = 0;
-  int krem = target;
-#pragma unroll 1
-  for (int shift = 56; shift >= 0; shift -= 8) {
+  // largest T_hi with #{hi >= T_hi} >= target (empty slots have hi = 0 and
+  // every real key has hi > 0)
+  uint32_t th = 0;
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t cand = th | (1u << b);
+    int c4[4] = {0, 0, 0, 0};   // independent partial counts
 #pragma unroll
-    for (int b = 0; b < 8; ++b) hist[lane * 8 + b] = 0;
-    __syncwarp();
-#pragma unroll
-    for (int k = 0; k < kSlots; ++k)
-      if (e[k] != 0ull && (e[k] & pmask) == prefix)
-        atomicAdd(&hist[static_cast<uint32_t>(e[k] >> shift) & 255u], 1u);
-    __syncwarp();
-    // lane l scans bins 255 - 8l down to 248 - 8l (descending digits)
-    uint32_t h[8], run = 0;
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      h[b] = hist[255 - (lane * 8 + b)];
-      run += h[b];
-    }
-    uint32_t incl = run;   // inclusive scan over lanes (higher digits first)
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const uint32_t excl = incl - run;
-    // the lane whose range holds the krem-th key (counting from the top)
-    const bool mine = excl < static_cast<uint32_t>(krem) && static_cast<uint32_t>(krem) <= incl;
-    const uint32_t owner = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-    uint32_t digit = 0, above = 0;
-    if (lane == owner) {
-      uint32_t acc = excl;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        if (acc + h[b] >= static_cast<uint32_t>(krem)) {
-          digit = 255 - (lane * 8 + b);
-          above = acc;
-          break;
-        }
-        acc += h[b];
-      }
-    }
-    digit = __shfl_sync(0xffffffffu, digit, owner);
-    above = __shfl_sync(0xffffffffu, above, owner);
-    krem -= static_cast<int>(above);
-    prefix |= static_cast<unsigned long long>(digit) << shift;
-    pmask |= 0xffull << shift;
-    __syncwarp();
+    for (int k = 0; k < kSlots; ++k) c4[k & 3] += hi[k] >= cand ? 1 : 0;
+    const int c = (c4[0] + c4[1]) + (c4[2] + c4[3]);
+    if (static_cast<int>(__reduce_add_sync(0xffffffffu, c)) >= target) th = cand;
   }
-  // prefix is now the exact target-th largest key: keep e >= prefix
+  int gt = 0, eq = 0;
+  uint32_t eq_min = 0xffffffffu;
+#pragma unroll
+  for (int k = 0; k < kSlots; ++k) {
+    gt += hi[k] > th ? 1 : 0;
+    if (hi[k] == th) {
+      ++eq;
+      eq_min = min(eq_min, lo[k]);
+    }
+  }
+  gt = static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+  eq = static_cast<int>(__reduce_add_sync(0xffffffffu, eq));
+  const int need = target - gt;   // 1 <= need <= eq
+  uint32_t tl;
+  if (need == eq) {
+    tl = __reduce_min_sync(0xffffffffu, eq_min);
+  } else {   // several keys share the score: the need-th largest token half among them
+    tl = 0;
+    for (int b = 31; b >= 0; --b) {
+      const uint32_t cand = tl | (1u << b);
+      int c = 0;
+#pragma unroll
+      for (int k = 0; k < kSlots; ++k) c += (hi[k] == th && lo[k] >= cand) ? 1 : 0;
+      if (static_cast<int>(__reduce_add_sync(0xffffffffu, c)) >= need) tl = cand;
+    }
+  }
+  const unsigned long long T = (static_cast<unsigned long long>(th) << 32) | tl;
   int out = 0;
 #pragma unroll
   for (int k = 0; k < kSlots; ++k) {
-    const bool keep = e[k] != 0ull && e[k] >= prefix;
+    const unsigned long long e = (static_cast<unsigned long long>(hi[k]) << 32) | lo[k];
+    const bool keep = hi[k] != 0u && e >= T;
     const uint32_t m = __ballot_sync(0xffffffffu, keep);
-    if (keep) buf[out + __popc(m & ((1u << lane) - 1u))] = e[k];
+    if (keep) buf[out + __popc(m & ((1u << lane) - 1u))] = e;
     out += __popc(m);
   }
   __syncwarp();
-  return prefix;
+  return T;
+}
+
+// v[c] for a run-time c in [0, 32) without a dynamic register index: a
+// five-level tree of selects on the bits of c.
+__device__ __forceinline__ float pick32(const float* v, int c) {
+  float a[16], b[8], d[4], e[2];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) a[k] = (c & 1) ? v[2 * k + 1] : v[2 * k];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) b[k] = (c & 2) ? a[2 * k + 1] : a[2 * k];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) d[k] = (c & 4) ? b[2 * k + 1] : b[2 * k];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) e[k] = (c & 8) ? d[2 * k + 1] : d[2 * k];
+  return (c & 16) ? e[1] : e[0];
 }
 
 template <int kCap>
@@ -223,7 +235,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kDBuf; ++b) {
       mbar_init(&ctl->d_full[b], 1);
       mbar_init(&ctl->d_empty[b], kBlock);
     }
@@ -269,9 +281,12 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       const uint32_t ahi = smem_u32(sm + kOffAhi), alo = smem_u32(sm + kOffAlo);
       bool ok = true;
       for (int it = 0; it < nblk && ok; ++it) {
-        const int stage = it % kSelRing, b = it & 1;
+        const int stage = it % kSelRing, b = it % kDBuf;
         if (!mbar_wait(&ctl->full[stage], (it / kSelRing) & 1, wc)) { ok = false; break; }
-        if (it >= 2 && !mbar_wait(&ctl->d_empty[b], ((it >> 1) - 1) & 1, wc)) { ok = false; break; }
+        if (it >= kDBuf && !mbar_wait(&ctl->d_empty[b], ((it / kDBuf) - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t kaddr = smem_u32(sm + kOffRingB + stage * kTileB);
         const uint32_t d = tmem + b * 128;
@@ -299,7 +314,6 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     const int r = tid;                        // query block i0 + r, TMEM lane r
     const bool live = r < rows;
     const int i = i0 + r;
-    uint32_t* scratch = &ctl->scratch[warp][0];
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int32_t* lrow = a.idx + (static_cast<size_t>(bh) * a.nb + (live ? i : i0)) * a.kcap;
     const int lcnt = live ? max(1, min(__ldg(a.cnt + static_cast<size_t>(bh) * a.nb + i), a.kcap)) : 0;
@@ -313,8 +327,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     bool ok = true;
     const int last_n = a.N - (a.nb - 1) * kBlock;
     for (int it = 0; it < nblk; ++it) {
-      const int j = a.pb + it, b = it & 1;
-      if (!sel_wait(&ctl->d_full[b], (it >> 1) & 1, wc)) { ok = false; break; }
+      const int j = a.pb + it, b = it % kDBuf;
+      if (!sel_wait(&ctl->d_full[b], (it / kDBuf) & 1, wc)) { ok = false; break; }
       tc_fence_after();
       float x[128];
       const uint32_t dcol = tmem + lane_base + b * 128;
@@ -330,27 +344,27 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         listed_j = true;
         ++cur;
       }
-      if (live && !listed_j) {
-        const int nvalid = (j == a.nb - 1) ? last_n : kBlock;
+      const bool scan = live && !listed_j;
+      const int nvalid = (j == a.nb - 1) ? last_n : kBlock;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t m = 0;
+      for (int q = 0; q < 4; ++q) {
+        uint32_t m = 0;
+        if (scan) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) m |= (x[32 * q + c] >= thf) ? (1u << c) : 0u;
           const int lim = nvalid - 32 * q;
           if (lim < 32) m &= lim > 0 ? ((1u << lim) - 1u) : 0u;
-          while (m) {
-            const int c = __ffs(m) - 1;
-            m &= m - 1;
-            // x[32q + c] without a dynamic register index
-            float xv = x[32 * q];
-#pragma unroll
-            for (int cc = 1; cc < 32; ++cc) xv = (cc == c) ? x[32 * q + cc] : xv;
-            const uint32_t u = static_cast<uint32_t>(j * kBlock + 32 * q + c);
-            const unsigned long long key =
-                (static_cast<unsigned long long>(orderable_key(xv)) << 32) | static_cast<uint32_t>(~u);
-            if (key > thr) buf[bcnt++] = key;
-          }
+        }
+        // every lane walks its own set bits: the lanes append together
+        while (m) {
+          const int c = __ffs(m) - 1;
+          m &= m - 1;
+          const float xv = pick32(x + 32 * q, c);
+          const uint32_t u = static_cast<uint32_t>(j * kBlock + 32 * q + c);
+          const unsigned long long key =
+              (static_cast<unsigned long long>(orderable_key(xv)) << 32) |
+              static_cast<uint32_t>(~u);
+          if (key > thr) buf[bcnt++] = key;
         }
       }
       // compact every full buffer of the warp, one row at a time
@@ -361,7 +375,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         unsigned long long* rb = reinterpret_cast<unsigned long long*>(
             __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(buf), L));
         const int count = __shfl_sync(0xffffffffu, bcnt, L);
-        const unsigned long long t = compact_keys<kSlots>(rb, count, a.n_extra, scratch);
+        const unsigned long long t = compact_keys<kSlots>(rb, count, a.n_extra);
         if (lane == L) {
           bcnt = a.n_extra;
           thr = t;
@@ -369,32 +383,9 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         }
       }
     }
-    // final: the n_extra largest (or all), written ascending by token
-    if (!ok) bcnt = 0;
-    for (int L = 0; L < 32; ++L) {
-      const int rL = warp * 32 + L;
-      if (rL >= rows) break;                   // uniform across the warp
-      unsigned long long* rb = reinterpret_cast<unsigned long long*>(
-          __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(buf), L));
-      int count = __shfl_sync(0xffffffffu, bcnt, L);
-      if (count > a.n_extra) {
-        compact_keys<kSlots>(rb, count, a.n_extra, scratch);
-        count = a.n_extra;
-      }
-      // tokens into the warp's scratch, then each lane ranks its entries
-      for (int p = lane; p < count; p += 32) scratch[p] = ~static_cast<uint32_t>(rb[p]);
-      __syncwarp();
-      int32_t* orow = a.extra + (static_cast<size_t>(bh) * a.nb + i0 + rL) * a.n_extra;
-      for (int p = lane; p < count; p += 32) {
-        const uint32_t u = scratch[p];
-        int rank = 0;
-        for (int q2 = 0; q2 < count; ++q2) rank += scratch[q2] < u ? 1 : 0;
-        orow[rank] = static_cast<int32_t>(u);
-      }
-      for (int p = count + lane; p < a.n_extra; p += 32) orow[p] = -1;
-      if (lane == 0) a.ecnt[static_cast<size_t>(bh) * a.nb + i0 + rL] = count;
-      __syncwarp();
-    }
+    // the buffer's fill count goes to the finishing kernel, which keeps the
+    // n_extra largest keys and writes them ascending by token
+    if (live) a.bcnt[static_cast<size_t>(bh) * a.nbv + (i - a.pb)] = ok ? bcnt : 0;
   }
 
   tc_fence_before();
@@ -404,6 +395,47 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kSelTmemCols);
   }
+}
+
+// One warp per video query block: the n_extra largest keys of its buffer (a
+// last compaction when more are left), written as tokens in ascending order
+// (each lane ranks its entries by counting smaller tokens in the warp's
+// shared buffer, four per 16-byte read), -1 padded; ecnt = their count.
+constexpr int kFinThreads = 256;
+
+template <int kCap>
+__global__ void __launch_bounds__(kFinThreads) extra_finish_kernel(const SelArgs a) {
+  __shared__ alignas(16) uint32_t sbuf[kFinThreads / 32][512 + 4];   // n_extra <= 512
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rowv = blockIdx.x * (kFinThreads / 32) + warp;   // video row over all heads
+  if (rowv >= a.rows_v) return;                               // whole warp
+  const int bh = rowv / a.nbv, i = a.pb + rowv % a.nbv;
+  unsigned long long* rb = a.cand + static_cast<size_t>(rowv) * kCap;
+  int count = max(0, min(__ldg(a.bcnt + rowv), kCap));
+  if (count > a.n_extra) {
+    compact_keys<kCap / 32>(rb, count, a.n_extra);
+    count = a.n_extra;
+  }
+  uint32_t* tok = sbuf[warp];
+  for (int p = lane; p < count; p += 32) tok[p] = ~static_cast<uint32_t>(rb[p]);
+  for (int p = count + lane; p < ((count + 3) & ~3); p += 32) tok[p] = 0xffffffffu;
+  __syncwarp();
+  int32_t* orow = a.extra + (static_cast<size_t>(bh) * a.nb + i) * a.n_extra;
+  const uint4* t4 = reinterpret_cast<const uint4*>(tok);
+  for (int p = lane; p < count; p += 32) {
+    const uint32_t u = tok[p];
+    int r4[4] = {0, 0, 0, 0};
+    for (int q4 = 0; q4 < (count + 3) / 4; ++q4) {
+      const uint4 t = t4[q4];
+      r4[0] += t.x < u ? 1 : 0;
+      r4[1] += t.y < u ? 1 : 0;
+      r4[2] += t.z < u ? 1 : 0;
+      r4[3] += t.w < u ? 1 : 0;
+    }
+    orow[(r4[0] + r4[1]) + (r4[2] + r4[3])] = static_cast<int32_t>(u);
+  }
+  for (int p = count + lane; p < a.n_extra; p += 32) orow[p] = -1;
+  if (lane == 0) a.ecnt[static_cast<size_t>(bh) * a.nb + i] = count;
 }
 
 // ------------------------------------------------------------------ side rows
@@ -436,15 +468,18 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__device__ __forceinline__ void load4(const __nv_bfloat16* p, float f[4]) {
-  const uint2 w = *reinterpret_cast<const uint2*>(p);
+
+__device__ __forceinline__ void bf16x4_to_f32(uint2 w, float f[4]) {
   f[0] = __uint_as_float(w.x << 16);
   f[1] = __uint_as_float(w.x & 0xffff0000u);
   f[2] = __uint_as_float(w.y << 16);
   f[3] = __uint_as_float(w.y & 0xffff0000u);
 }
 
-__global__ void __launch_bounds__(kSumThreads) extra_summary_kernel(const SideArgs a) {
+// One CTA (4 warps) per video query block; each warp takes runs of tokens of
+// one block (lane l: dimensions 4l..4l+3), gathering each token's K and V row
+// once: its anchor logit (a warp sum), its weight and its share of the sums.
+__global__ void __launch_bounds__(kSumThreads, 8) extra_summary_kernel(const SideArgs a) {
   __shared__ int32_t toks[512];
   __shared__ int32_t seg_start[513];
   __shared__ int32_t seg_row[513];
@@ -453,35 +488,43 @@ __global__ void __launch_bounds__(kSumThreads) extra_summary_kernel(const SideAr
   const int i = a.pb + blockIdx.x;
   const size_t bh = blockIdx.y;
   const size_t row_id = bh * a.nb + i;
-  const int m = max(0, min(__ldg(a.ecnt + row_id), a.n_extra));
-  for (int p = tid; p < m; p += kSumThreads) toks[p] = __ldg(a.extra + row_id * a.n_extra + p);
+  const int m_in = max(0, min(__ldg(a.ecnt + row_id), a.n_extra));
+  const bool anchor_variant = a.variant == 0;
+  for (int p = tid; p < m_in; p += kSumThreads) toks[p] = __ldg(a.extra + row_id * a.n_extra + p);
   __syncthreads();
   if (tid == 0) {
+    // the list is used up to its first token that is not a video token or
+    // not above its predecessor (a valid list has none), so every row read
+    // below lies inside the head
+    int m = 0;
+    while (m < m_in && toks[m] >= a.pb * kBlock && toks[m] < a.N &&
+           (m == 0 || toks[m] > toks[m - 1]))
+      ++m;
     // runs of equal block; a run covering a whole block leaves no row
     int ns = 0, nr = 0;
     for (int p = 0; p < m; ++p) {
-      if (p == 0 || (toks[p] >> 7) != (toks[p - 1] >> 7)) {
-        seg_start[ns] = p;
-        ++ns;
-      }
+      if (p == 0 || (toks[p] >> 7) != (toks[p - 1] >> 7)) seg_start[ns++] = p;
     }
     seg_start[ns] = m;
     for (int s = 0; s < ns; ++s) {
       const int j = toks[seg_start[s]] >> 7;
       const int nj = min(kBlock, a.N - j * kBlock);
-      const int e = seg_start[s + 1] - seg_start[s];
-      seg_row[s] = (e < nj) ? nr++ : -1;
+      seg_row[s] = (seg_start[s + 1] - seg_start[s] < nj) ? nr++ : -1;
     }
     nseg_s = ns;
     nrow_s = nr;
   }
   __syncthreads();
   const int nseg = nseg_s, nrow = nrow_s;
-  const float* qbar = a.anchor + bh * kDim;
-  float qb[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) qb[k] = __ldg(qbar + 4 * lane + k);
   const size_t side_row0 = row_id * a.scap;
+  float q4[4] = {0.f, 0.f, 0.f, 0.f};
+  if (anchor_variant) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(a.anchor + bh * kDim) + lane);
+    q4[0] = t.x; q4[1] = t.y; q4[2] = t.z; q4[3] = t.w;
+  }
+  auto logit = [&](const float kf[4]) {
+    return warp_sum(q4[0] * kf[0] + q4[1] * kf[1] + q4[2] * kf[2] + q4[3] * kf[3]) * a.scale;
+  };
 
   for (int s = warp; s < nseg; s += kSumThreads / 32) {
     const int row = seg_row[s];
@@ -491,17 +534,15 @@ __global__ void __launch_bounds__(kSumThreads) extra_summary_kernel(const SideAr
     const int nj = min(kBlock, a.N - j * kBlock);
     const size_t blk = bh * a.nb + j;
     float kn[4], vn[4], Lnew;
-    if (a.variant == 0) {
+    if (anchor_variant) {
       const float L = __ldg(a.lse_blk + blk);
       float sw = 0.f, swk[4] = {0.f, 0.f, 0.f, 0.f}, swv[4] = {0.f, 0.f, 0.f, 0.f};
       for (int p = p0; p < p1; ++p) {
         const size_t t = bh * a.N + toks[p];
         float kf[4], vf[4];
-        load4(a.K + t * kDim + 4 * lane, kf);
-        load4(a.V + t * kDim + 4 * lane, vf);
-        const float x = warp_sum(qb[0] * kf[0] + qb[1] * kf[1] + qb[2] * kf[2] + qb[3] * kf[3]) *
-                        a.scale;
-        const float w = expf(x - L);
+        bf16x4_to_f32(*reinterpret_cast<const uint2*>(a.K + t * kDim + 4 * lane), kf);
+        bf16x4_to_f32(*reinterpret_cast<const uint2*>(a.V + t * kDim + 4 * lane), vf);
+        const float w = expf(logit(kf) - L);
         sw += w;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -512,11 +553,12 @@ __global__ void __launch_bounds__(kSumThreads) extra_summary_kernel(const SideAr
       const float R = 1.f - sw;
       if (R >= kDowndateMin) {
         const float invR = 1.f / R;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          kn[k] = (__ldg(a.kstat + blk * kDim + 4 * lane + k) - swk[k]) * invR;
-          vn[k] = (__ldg(a.vstat + blk * kDim + 4 * lane + k) - swv[k]) * invR;
-        }
+        const float4 ks4 = __ldg(reinterpret_cast<const float4*>(a.kstat + blk * kDim) + lane);
+        const float4 vs4 = __ldg(reinterpret_cast<const float4*>(a.vstat + blk * kDim) + lane);
+        kn[0] = (ks4.x - swk[0]) * invR; kn[1] = (ks4.y - swk[1]) * invR;
+        kn[2] = (ks4.z - swk[2]) * invR; kn[3] = (ks4.w - swk[3]) * invR;
+        vn[0] = (vs4.x - swv[0]) * invR; vn[1] = (vs4.y - swv[1]) * invR;
+        vn[2] = (vs4.z - swv[2]) * invR; vn[3] = (vs4.w - swv[3]) * invR;
         Lnew = L + logf(R);
       } else {
         // recompute over the remaining rows (max-subtracted sums)
@@ -530,10 +572,9 @@ __global__ void __launch_bounds__(kSumThreads) extra_summary_kernel(const SideAr
           }
           const size_t t = bh * a.N + u;
           float kf[4], vf[4];
-          load4(a.K + t * kDim + 4 * lane, kf);
-          load4(a.V + t * kDim + 4 * lane, vf);
-          const float x = warp_sum(qb[0] * kf[0] + qb[1] * kf[1] + qb[2] * kf[2] + qb[3] * kf[3]) *
-                          a.scale;
+          bf16x4_to_f32(*reinterpret_cast<const uint2*>(a.K + t * kDim + 4 * lane), kf);
+          bf16x4_to_f32(*reinterpret_cast<const uint2*>(a.V + t * kDim + 4 * lane), vf);
+          const float x = logit(kf);
           const float mn = fmaxf(mx, x);
           const float f = expf(mx - mn), w = expf(x - mn);
           ssum = ssum * f + w;
@@ -557,8 +598,8 @@ __global__ void __launch_bounds__(kSumThreads) extra_summary_kernel(const SideAr
       for (int p = p0; p < p1; ++p) {
         const size_t t = bh * a.N + toks[p];
         float kf[4], vf[4];
-        load4(a.K + t * kDim + 4 * lane, kf);
-        load4(a.V + t * kDim + 4 * lane, vf);
+        bf16x4_to_f32(*reinterpret_cast<const uint2*>(a.K + t * kDim + 4 * lane), kf);
+        bf16x4_to_f32(*reinterpret_cast<const uint2*>(a.V + t * kDim + 4 * lane), vf);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           sk[k] += kf[k];
@@ -566,12 +607,12 @@ __global__ void __launch_bounds__(kSumThreads) extra_summary_kernel(const SideAr
         }
       }
       const float n = static_cast<float>(nj), rest = static_cast<float>(nj - (p1 - p0));
-      const float inv = 1.f / rest;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        kn[k] = (n * __ldg(a.kpool + blk * kDim + 4 * lane + k) - sk[k]) * inv;
-        vn[k] = (n * __ldg(a.vstat + blk * kDim + 4 * lane + k) - sv[k]) * inv;
-      }
+      const float4 kp4 = __ldg(reinterpret_cast<const float4*>(a.kpool + blk * kDim) + lane);
+      const float4 vs4 = __ldg(reinterpret_cast<const float4*>(a.vstat + blk * kDim) + lane);
+      kn[0] = (n * kp4.x - sk[0]) / rest; kn[1] = (n * kp4.y - sk[1]) / rest;
+      kn[2] = (n * kp4.z - sk[2]) / rest; kn[3] = (n * kp4.w - sk[3]) / rest;
+      vn[0] = (n * vs4.x - sv[0]) / rest; vn[1] = (n * vs4.y - sv[1]) / rest;
+      vn[2] = (n * vs4.z - sv[2]) / rest; vn[3] = (n * vs4.w - sv[3]) / rest;
       Lnew = logf(rest);
     }
     // bf16 rows as the MMA will read them; the anchor bias from bf16(k~')
@@ -581,10 +622,10 @@ __global__ void __launch_bounds__(kSumThreads) extra_summary_kernel(const SideAr
     vw.x = pack_bf16x2(vn[0], vn[1]);
     vw.y = pack_bf16x2(vn[2], vn[3]);
     float bias = Lnew;
-    if (a.variant == 0) {
-      const float dot = qb[0] * bf16_round(kn[0]) + qb[1] * bf16_round(kn[1]) +
-                        qb[2] * bf16_round(kn[2]) + qb[3] * bf16_round(kn[3]);
-      bias = Lnew - warp_sum(dot) * a.scale;
+    if (anchor_variant) {
+      float kb[4];
+      bf16x4_to_f32(kw, kb);
+      bias = Lnew - logit(kb);
     }
     const size_t o = side_row0 + row;
     *reinterpret_cast<uint2*>(a.side_k + o * kDim + 4 * lane) = kw;
@@ -621,16 +662,19 @@ cudaError_t launch_select_extra_t(const Shape& s, const CUtensorMap& tm_k, const
   if (e != cudaSuccess) return e;
   const dim3 grid((s.nbv + kBlock - 1) / kBlock, s.B * s.H);
   select_extra_kernel<kCap><<<grid, kSelThreads, smem, st>>>(tm_k, a);
+  const int fgrid = (a.rows_v + kFinThreads / 32 - 1) / (kFinThreads / 32);
+  extra_finish_kernel<kCap><<<fgrid, kFinThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int extra_cand_cap(int n_extra) { return n_extra <= 256 ? 768 : 1280; }
+int extra_cand_cap(int n_extra) { return n_extra <= 256 ? 1280 : 2048; }
 
 size_t select_extra_scratch_bytes(const Shape& s, int n_extra) {
   if (n_extra <= 0) return 0;
-  return static_cast<size_t>(s.B) * s.H * s.nbv * extra_cand_cap(n_extra) * 8;
+  const size_t rows = static_cast<size_t>(s.B) * s.H * s.nbv;
+  return rows * extra_cand_cap(n_extra) * 8 + rows * 4;   // buffers, then their fill counts
 }
 
 int extra_side_cap(const Shape& s, int n_extra) {
@@ -647,6 +691,9 @@ cudaError_t launch_select_extra(const Shape& s, int n_extra, const CUtensorMap& 
   a.idx = idx;
   a.cnt = cnt;
   a.cand = static_cast<unsigned long long*>(scratch);
+  a.rows_v = s.B * s.H * s.nbv;
+  a.bcnt = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) +
+                                      static_cast<size_t>(a.rows_v) * extra_cand_cap(n_extra) * 8);
   a.extra = extra;
   a.ecnt = ecnt;
   a.dev_status = s.dev_status;
@@ -656,8 +703,8 @@ cudaError_t launch_select_extra(const Shape& s, int n_extra, const CUtensorMap& 
   a.nbv = s.nbv;
   a.kcap = kcap;
   a.n_extra = n_extra;
-  return extra_cand_cap(n_extra) == 768 ? launch_select_extra_t<768>(s, tm_k, a, st)
-                                        : launch_select_extra_t<1280>(s, tm_k, a, st);
+  return extra_cand_cap(n_extra) == 1280 ? launch_select_extra_t<1280>(s, tm_k, a, st)
+                                         : launch_select_extra_t<2048>(s, tm_k, a, st);
 }
 
 cudaError_t launch_extra_summaries(const Shape& s, int n_extra, const void* K, const void* V,

@@ -4,11 +4,11 @@
 // One CTA per (tile of R query blocks, head), 256 threads:
 //  1. scores  S_ij = qpool_i . kpool_j / sqrt(128) in fp32 for every video
 //     key block j >= pb, kept in shared memory (never written to HBM).  The
-//     pooled keys stream through shared memory 32 blocks at a time
+//     pooled keys stream through shared memory 128 blocks at a time
 //     (coalesced 16-byte loads, rows padded against bank conflicts); each
-//     thread forms the dot products of two query blocks with one key block
-//     with packed fp32x2 FMAs (even and odd dimensions in two partial sums,
-//     added at the end; a fixed order, so the result is deterministic).
+//     thread forms the dot products of four query blocks with four key
+//     blocks with packed fp32x2 FMAs (even and odd dimensions in two partial
+//     sums, added at the end; a fixed order, so the result is deterministic).
 //  2. one warp per query block finds the k_eff-th largest score as a 32-bit
 //     order-preserving key by bitwise binary search (32 count passes,
 //     __reduce_add_sync per pass, the row's keys held in registers), then
@@ -31,7 +31,7 @@ namespace bsa {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 32;               // key blocks per shared-memory chunk
+constexpr int kChunk = 128;              // key blocks per shared-memory chunk
 constexpr int kPad = kDim + 4;           // padded row of 132 floats
 
 // Top-k of one row of nbv scores (in shared memory) by warp `lane`s; the keys
@@ -190,9 +190,12 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float* __restric
       *reinterpret_cast<float4*>(qp + r * kPad + 4 * d4) =
           __ldg(reinterpret_cast<const float4*>(qpool + (bh * nb + i) * kDim) + d4);
     }
-    // thread -> (query-block pair rp, key k of the chunk); R/2 pairs x 32 keys
-    const int pairs = R / 2;
-    const int rp = tid / kChunk, kk = tid % kChunk;
+    // thread -> 4 query blocks (rows 4*warp .. 4*warp+3) x 4 key blocks of the
+    // chunk (lane, lane+32, lane+64, lane+96): 16 dot products per thread, so
+    // each 16-byte shared load feeds four of them.  Every dot product keeps
+    // even and odd dimensions in two partial sums added at the end (a fixed
+    // order: the result is deterministic).
+    const int rg = warp;   // row group
     for (int c0 = 0; c0 < nbv; c0 += kChunk) {
       __syncthreads();   // previous chunk fully used (and qp written, first time)
       const int rows = min(kChunk, nbv - c0);
@@ -202,23 +205,39 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float* __restric
             reinterpret_cast<const float4*>(kpool + (bh * nb + pb + c0 + r) * kDim) + d4);
       }
       __syncthreads();
-      if (rp < pairs && kk < rows) {
-        const float* q0 = qp + (2 * rp) * kPad;
-        const float* q1 = q0 + kPad;
-        const float* kr = kc + kk * kPad;
-        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
-#pragma unroll 8
+      if (4 * rg < R) {
+        float2 acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] = make_float2(0.f, 0.f);
+        const float* q0 = qp + (4 * rg) * kPad;
+#pragma unroll 4
         for (int d4 = 0; d4 < kDim / 4; ++d4) {
-          const float4 k4 = *reinterpret_cast<const float4*>(kr + 4 * d4);
-          const float4 x0 = *reinterpret_cast<const float4*>(q0 + 4 * d4);
-          const float4 x1 = *reinterpret_cast<const float4*>(q1 + 4 * d4);
-          a0 = fma2(make_float2(x0.x, x0.y), make_float2(k4.x, k4.y), a0);
-          a0 = fma2(make_float2(x0.z, x0.w), make_float2(k4.z, k4.w), a0);
-          a1 = fma2(make_float2(x1.x, x1.y), make_float2(k4.x, k4.y), a1);
-          a1 = fma2(make_float2(x1.z, x1.w), make_float2(k4.z, k4.w), a1);
+          float4 x[4], k[4];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) x[a] = *reinterpret_cast<const float4*>(q0 + a * kPad + 4 * d4);
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            k[b] = *reinterpret_cast<const float4*>(kc + (lane + 32 * b) * kPad + 4 * d4);
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              acc[a][b] = fma2(make_float2(x[a].x, x[a].y), make_float2(k[b].x, k[b].y), acc[a][b]);
+              acc[a][b] = fma2(make_float2(x[a].z, x[a].w), make_float2(k[b].z, k[b].w), acc[a][b]);
+            }
         }
-        sc[(2 * rp) * nbv + c0 + kk] = (a0.x + a0.y) * scale;
-        sc[(2 * rp + 1) * nbv + c0 + kk] = (a1.x + a1.y) * scale;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const int r = 4 * rg + a;
+          if (r >= R) break;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int kk = lane + 32 * b;
+            if (kk < rows) sc[r * nbv + c0 + kk] = (acc[a][b].x + acc[a][b].y) * scale;
+          }
+        }
       }
     }
     __syncthreads();
@@ -253,7 +272,7 @@ cudaError_t launch_select_t(const Shape& s, const float* qpool, const float* kpo
   static std::atomic<bool> attr_set[64];
   cudaError_t e = once_per_device(attr_set, [] {
     return cudaFuncSetAttribute(select_kernel<kPerLane, kThresh>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
   });
   if (e != cudaSuccess) return e;
   const dim3 grid((s.nb + R - 1) / R, s.B * s.H);
@@ -267,12 +286,16 @@ cudaError_t launch_select_t(const Shape& s, const float* qpool, const float* kpo
 
 }  // namespace
 
-// Query blocks per CTA: 16 (an even number, so the pair mapping covers it),
-// fewer when a row of scores is long, so the tile stays within ~180 KB.
+// Query blocks per CTA: 16 for rows of fewer than 512 blocks (two CTAs fit
+// on an SM), else 32 (four per warp in the score phase: each chunk of pooled
+// keys serves twice the rows); fewer when a row of scores is long, so the
+// tile stays within the shared memory of one CTA (at least one row: N <=
+// 2^21 keeps a row under 64 KB).  Measured at 56 heads: 0.113 against 0.149
+// ms with 16 and 32 rows at 295 blocks, 1.29 against 1.13 ms at 1045.
 static int select_rows(int nbv) {
   const size_t fixed = static_cast<size_t>(kChunk) * kPad * 4;
-  int R = 16;
-  while (R > 2 && fixed + static_cast<size_t>(R) * (kPad + nbv) * 4 > 180 * 1024) R -= 2;
+  int R = nbv < 512 ? 16 : 32;
+  while (R > 1 && fixed + static_cast<size_t>(R) * (kPad + nbv) * 4 > 220 * 1024) --R;
   return R;
 }
 
