@@ -133,8 +133,23 @@ def forward_head_fp8(Q, K, V, top_k: int, prefix: int = 0, variant: str = "ancho
                 vs_scale=svs, Qd=Qd, Kd=Kd, Vd=Vd, KSd=KSd, VSd=VSd, O=O, lse=lse)
 
 
+def weight_moves(p, r, exp_rel_err: float = 0.0):
+    """Largest move of each softmax weight w = p / sum(p) (last axis) when the
+    kernel rounds p * r to e4m3 (r = s_v / s_ref <= 1) after computing p with
+    relative error at most ``exp_rel_err`` = e, and divides by the sum of its
+    own numerators: max(rho w, 2^-10 / (r l (1 - e)) + w 2e / (1 - e)) with
+    rho = (1 + e)(1 + 2^-4) / (1 - e) - 1 and l = sum(p) (see
+    fp8_output_bound for the derivation)."""
+    p = np.asarray(p, dtype=np.float64)
+    l = p.sum(axis=-1, keepdims=True)
+    e = float(exp_rel_err)
+    rho = (1 + e) * (1 + 2.0 ** -4) / (1 - e) - 1
+    return np.maximum(rho * p / l, 2.0 ** -10 / (r * l * (1 - e)) + (2 * e / (1 - e)) * p / l)
+
+
 def fp8_output_bound(Qd, Kd, Vd, lists, KSd, VSd, bias, v_scale, vs_scale, prefix_blocks: int,
-                     block: int = BLOCK, query_blocks=None, with_variance: bool = False):
+                     block: int = BLOCK, query_blocks=None, with_variance: bool = False,
+                     exp_rel_err: float = 0.0):
     """Per-element bound on |O_kernel - O| from the kernel's e4m3 numerators.
 
     The kernel writes each softmax numerator p (relative to a running max at
@@ -145,6 +160,14 @@ def fp8_output_bound(Qd, Kd, Vd, lists, KSd, VSd, bias, v_scale, vs_scale, prefi
     column's weight moves by at most max(2^-4 w, 2^-10 / (r * l)), with w the
     exact weight and l = sum_t exp(x_t - max) the exact row sum.  The bound is
     the sum of those moves times |v|, column by column.
+
+    ``exp_rel_err`` = e: the kernel's numerators before rounding are
+    p (1 + e_t) with |e_t| <= e (an approximate exponential), and its row sum
+    is the sum of those, l (1 + e_l) with |e_l| <= e.  Then a normal code's
+    weight is w (1 + e_t)(1 + d_t) / (1 + e_l) with |d_t| <= 2^-4, which moves
+    by at most rho w, rho = (1 + e)(1 + 2^-4) / (1 - e) - 1; a subnormal
+    code's by at most 2^-10 / (r l (1 - e)) + w (2 e / (1 - e)).  With e = 0
+    both reduce to the moves above.
 
     With ``with_variance`` it also returns an upper model of each element's
     error variance: rounding to nearest leaves an error spread over at most
@@ -178,8 +201,7 @@ def fp8_output_bound(Qd, Kd, Vd, lists, KSd, VSd, bias, v_scale, vs_scale, prefi
                 r = np.concatenate([r, np.array([vs_scale[j // block] for j in skipped]) / s_ref])
         m = logits.max(axis=1, keepdims=True)
         p = np.exp(logits - m)
-        l = p.sum(axis=1, keepdims=True)
-        move = np.maximum(2.0 ** -4 * p / l, 2.0 ** -10 / (r[None, :] * l))
+        move = weight_moves(p, r[None, :], exp_rel_err)
         out[a:b] = move @ vals
         var[a:b] = (move ** 2 / 3) @ (vals ** 2)
     return (out, var) if with_variance else out

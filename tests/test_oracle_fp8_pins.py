@@ -184,3 +184,76 @@ def test_output_bound_needs_its_subnormal_term():
         rel_only = (2.0 ** -4 * p / l) @ np.abs(r8["Vd"][tok])
         rel_only_violated |= bool((err > rel_only + 1e-12).any())
     assert rel_only_violated
+
+
+def test_output_bound_covers_approximate_exponentials():
+    # The kernel may compute some softmax numerators with an approximate
+    # exponential: p (1 + e_t), |e_t| <= e, and sums those into its row sum.
+    # Simulated with the worst signs (alternating +e and -e per column, and
+    # all +e or all -e), the bound with exp_rel_err = e holds element by
+    # element.
+    rng = np.random.default_rng(7)
+    N, d, top_k = 600, 8, 2
+    Q = rng.standard_normal((N, d)) * 1.5
+    K = rng.standard_normal((N, d)) * 1.5
+    V = rng.standard_normal((N, d))
+    r8 = f8.forward_head_fp8(Q, K, V, top_k, 0)
+    eps = 2.0 ** -6
+    args = (r8["Qd"], r8["Kd"], r8["Vd"], r8["lists"], r8["KSd"], r8["VSd"], r8["bias"],
+            r8["v_scale"], r8["vs_scale"], 0)
+    bound_e = f8.fp8_output_bound(*args, exp_rel_err=eps)
+    bound_0 = f8.fp8_output_bound(*args)
+    s_ref = max(r8["v_scale"].max(), r8["vs_scale"].max())
+    bounds = orc.block_bounds(N)
+    nb = len(bounds)
+    for pattern in ("alternate", "plus", "minus"):
+        for i, (a, b) in enumerate(bounds):
+            E = [int(j) for j in r8["lists"][i]]
+            tok = np.concatenate([np.arange(*bounds[j]) for j in E])
+            sk = [j for j in range(nb) if j not in E]
+            logits = np.concatenate([r8["Qd"][a:b] @ r8["Kd"][tok].T / np.sqrt(d),
+                                     r8["Qd"][a:b] @ r8["KSd"][sk].T / np.sqrt(d)
+                                     + r8["bias"][sk]], axis=1)
+            vcodes = np.concatenate([r8["v_codes"][tok], r8["vs_codes"][sk]])
+            r = np.concatenate([r8["v_scale"][tok // 128],
+                                r8["vs_scale"][np.array(sk) // 128]]) / s_ref
+            p = np.exp(logits - logits.max(axis=1, keepdims=True))
+            sign = {"alternate": np.where(np.arange(p.shape[1]) % 2 == 0, 1.0, -1.0),
+                    "plus": np.ones(p.shape[1]), "minus": -np.ones(p.shape[1])}[pattern]
+            pt = p * (1 + eps * sign[None, :])
+            O_sim = s_ref * (f8.round_e4m3(pt * r[None, :]) @ vcodes) / pt.sum(axis=1,
+                                                                           keepdims=True)
+            err = np.abs(O_sim - r8["O"][a:b])
+            assert (err <= bound_e[a:b] + 1e-12).all(), (pattern, i)
+    assert (bound_e >= bound_0).all() and (bound_e > bound_0).any()
+
+
+def test_weight_moves_need_the_approximate_exponential_term():
+    # Brute force over rows of numerators, e4m3 rounding and the kernel's own
+    # row sum: every weight stays within weight_moves(e).  A constructed row
+    # where one numerator sits just below a rounding midpoint (so e4m3 rounds
+    # it down by almost 2^-4) and is pushed down by -e while the others are
+    # pushed up (so the row sum grows) moves further than the bound without
+    # the term allows.
+    rng = np.random.default_rng(8)
+    eps = 2.0 ** -5
+    for _ in range(200):
+        n = 64
+        p = np.exp(-rng.exponential(3.0, n))
+        p[rng.integers(n)] = 1.0
+        r = rng.uniform(0.2, 1.0, n)
+        et = rng.choice([-eps, eps], n)
+        pt = p * (1 + et)
+        w_hat = f8.round_e4m3(pt * r) / (r * pt.sum())
+        w = p / p.sum()
+        assert (np.abs(w_hat - w) <= f8.weight_moves(p, r, eps) + 1e-15).all()
+    # the constructed row
+    k = 1.0 + 2.0 ** -4 - 2.0 ** -11          # rounds down to 1.0 in e4m3
+    p = np.array([k / (1 - eps), 1.0, 1.0, 1.0])
+    r = np.ones(4)
+    pt = p * np.array([1 - eps, 1 + eps, 1 + eps, 1 + eps])
+    assert f8.round_e4m3(np.array([pt[0]]))[0] == 1.0
+    w_hat = f8.round_e4m3(pt * r) / (r * pt.sum())
+    w = p / p.sum()
+    assert abs(w_hat[0] - w[0]) <= f8.weight_moves(p, r, eps)[0]
+    assert abs(w_hat[0] - w[0]) > f8.weight_moves(p, r, 0.0)[0]
