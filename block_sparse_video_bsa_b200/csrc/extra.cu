@@ -65,6 +65,9 @@ struct SelCtl {
   uint32_t tmem_base;
   int abort_flag;
   int skip;
+  // per selection warp: the 32 scores of a column group of every lane, [column][lane],
+  // read back by the lanes' appends
+  float xs[4][32][32];
 };
 static_assert(kOffSelCtl + sizeof(SelCtl) <= 227 * 1024, "shared memory budget");
 
@@ -166,21 +169,6 @@ __device__ unsigned long long compact_keys(unsigned long long* buf, int count, i
   }
   __syncwarp();
   return T;
-}
-
-// v[c] for a run-time c in [0, 32) without a dynamic register index: a
-// five-level tree of selects on the bits of c.
-__device__ __forceinline__ float pick32(const float* v, int c) {
-  float a[16], b[8], d[4], e[2];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) a[k] = (c & 1) ? v[2 * k + 1] : v[2 * k];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) b[k] = (c & 2) ? a[2 * k + 1] : a[2 * k];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) d[k] = (c & 4) ? b[2 * k + 1] : b[2 * k];
-#pragma unroll
-  for (int k = 0; k < 2; ++k) e[k] = (c & 8) ? d[2 * k + 1] : d[2 * k];
-  return (c & 16) ? e[1] : e[0];
 }
 
 template <int kCap>
@@ -325,6 +313,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     unsigned long long thr = 0ull;
     float thf = -INFINITY;
     bool ok = true;
+    float (*xsw)[32] = ctl->xs[warp];
     const int last_n = a.N - (a.nb - 1) * kBlock;
     for (int it = 0; it < nblk; ++it) {
       const int j = a.pb + it, b = it % kDBuf;
@@ -355,11 +344,18 @@ __global__ void __launch_bounds__(kSelThreads, 1)
           const int lim = nvalid - 32 * q;
           if (lim < 32) m &= lim > 0 ? ((1u << lim) - 1u) : 0u;
         }
-        // every lane walks its own set bits: the lanes append together
+        // every lane walks its own set bits: the lanes append together, each
+        // reading its score back from the warp's copy of the group
+        if (__any_sync(0xffffffffu, m != 0)) {
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) xsw[c][lane] = x[32 * q + c];
+          __syncwarp();
+        }
         while (m) {
           const int c = __ffs(m) - 1;
           m &= m - 1;
-          const float xv = pick32(x + 32 * q, c);
+          const float xv = xsw[c][lane];
           const uint32_t u = static_cast<uint32_t>(j * kBlock + 32 * q + c);
           const unsigned long long key =
               (static_cast<unsigned long long>(orderable_key(xv)) << 32) |
