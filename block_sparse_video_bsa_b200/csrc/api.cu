@@ -125,6 +125,35 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t BH) {
          CUDA_SUCCESS;
 }
 
+// fp32 [BH, rows, 128] viewed as a 3-D tensor; box = 32 columns (128 bytes,
+// one swizzle atom) x box_rows rows x 1 head.  Rows past `rows` read as zero.
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t BH,
+                  uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {128, rows, BH};
+  const cuuint64_t strides[2] = {128 * 4, rows * 128 * 4};
+  const cuuint32_t box[3] = {32, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// The pooled-score maps of the tensor-core selection, or NULL when the rows
+// are too long for it (the SIMT kernel then runs) or a map cannot be made.
+const bsa::SelectMaps* select_maps(const Shape& s, const float* qpool, const float* kpool,
+                                   bsa::SelectMaps* m) {
+  const int R = bsa::select_tc_rows(s);
+  if (R <= 0) return nullptr;
+  const uint64_t bh = static_cast<uint64_t>(s.B) * s.H;
+  if (!make_map_f32(&m->q, qpool, s.nb, bh, static_cast<uint32_t>(R)) ||
+      !make_map_f32(&m->k, kpool, s.nb, bh, 128))
+    return nullptr;
+  return m;
+}
+
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // The FP8 operand set carved from one buffer in the order of
@@ -231,7 +260,9 @@ int summarize_impl(const Shape& s, const void* K, const void* V, const float* an
 }
 int select_impl(const Shape& s, const float* qpool, const float* kpool, int32_t* idx, int32_t* cnt,
                 cudaStream_t st) {
-  return cuda_status(bsa::launch_select(s, qpool, kpool, idx, cnt, st));
+  bsa::SelectMaps m;
+  return cuda_status(bsa::launch_select(s, select_maps(s, qpool, kpool, &m), qpool, kpool, idx,
+                                        cnt, st));
 }
 int attend_impl(const Shape& s, const void* Q, const void* K, const void* V, const int32_t* idx,
                 const int32_t* cnt, const void* ksum, const void* vsum, const float* bias, void* O,
@@ -895,7 +926,9 @@ int bsa_select_threshold(const bsa_params* p, float tau, const float* qpool, con
   if (!aligned(qpool, 16) || !aligned(kpool, 16) || !aligned(idx, 4) || !aligned(cnt, 4))
     return BSA_ERR_ALIGN;
   if ((rc = check_device())) return rc;
-  return cuda_status(bsa::launch_select_threshold(s, tau, qpool, kpool, idx, cnt,
+  bsa::SelectMaps m;
+  return cuda_status(bsa::launch_select_threshold(s, tau, select_maps(s, qpool, kpool, &m), qpool,
+                                                  kpool, idx, cnt,
                                                   static_cast<cudaStream_t>(stream)));
 }
 
@@ -951,7 +984,9 @@ int bsa_forward_threshold(const bsa_params* p, float tau, const void* Q, const v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = pool_impl(s, Q, w.qpool, w.anchor, st))) return rc;
   if ((rc = summarize_impl(s, K, V, w.anchor, w.kpool, w.ksum, w.vsum, w.bias, st))) return rc;
-  if ((rc = cuda_status(bsa::launch_select_threshold(s, tau, w.qpool, w.kpool, w.idx, w.cnt, st))))
+  bsa::SelectMaps m;
+  if ((rc = cuda_status(bsa::launch_select_threshold(
+           s, tau, select_maps(s, w.qpool, w.kpool, &m), w.qpool, w.kpool, w.idx, w.cnt, st))))
     return rc;
   return attend_lists_impl(s, Q, K, V, w.idx, s.nb, w.cnt, w.ksum, w.vsum, w.bias, O, lse,
                            static_cast<uint8_t*>(workspace) + ws0, st);

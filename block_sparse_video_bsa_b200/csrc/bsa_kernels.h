@@ -47,12 +47,20 @@ cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const
                              float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st,
                              float* kstat = nullptr, float* vstat = nullptr,
                              float* lse_blk = nullptr);
-cudaError_t launch_select(const Shape& s, const float* qpool, const float* kpool, int32_t* idx,
-                          int32_t* cnt, cudaStream_t st);
+// Selection.  With `maps` (fp32 qpool / kpool as [BH, nb, 128] with 128-byte
+// swizzle, boxes {32, select_tc_rows(s), 1} and {32, 128, 1}) and
+// select_tc_rows(s) > 0 the scores come from the tensor cores; otherwise
+// (maps NULL, or rows too long for TMEM) from the SIMT kernel.
+int select_tc_rows(const Shape& s);
+struct SelectMaps {
+  CUtensorMap q, k;
+};
+cudaError_t launch_select(const Shape& s, const SelectMaps* maps, const float* qpool,
+                          const float* kpool, int32_t* idx, int32_t* cnt, cudaStream_t st);
 // Threshold selection: idx rows of length nb (kcap ignored), cnt per row.
-cudaError_t launch_select_threshold(const Shape& s, float tau, const float* qpool,
-                                    const float* kpool, int32_t* idx, int32_t* cnt,
-                                    cudaStream_t st);
+cudaError_t launch_select_threshold(const Shape& s, float tau, const SelectMaps* maps,
+                                    const float* qpool, const float* kpool, int32_t* idx,
+                                    int32_t* cnt, cudaStream_t st);
 
 struct AttendMaps {
   CUtensorMap q, k, v, ks, vs;   // bf16, box {64, 128, 1}, 128B swizzle
