@@ -49,8 +49,9 @@ cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const
                              float* lse_blk = nullptr);
 // Selection.  With `maps` (fp32 qpool / kpool as [BH, nb, 128] with 128-byte
 // swizzle, boxes {32, select_tc_rows(s), 1} and {32, 128, 1}) and
-// select_tc_rows(s) > 0 the scores come from the tensor cores; otherwise
-// (maps NULL, or rows too long for TMEM) from the SIMT kernel.
+// select_tc_rows(s) > 0 (rows of up to 3072 video blocks) the scores come
+// from the tensor cores; otherwise (maps NULL, or longer rows) from the SIMT
+// kernel.
 int select_tc_rows(const Shape& s);
 struct SelectMaps {
   CUtensorMap q, k;

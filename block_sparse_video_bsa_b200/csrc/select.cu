@@ -17,9 +17,9 @@
 //     the lower index".
 // Dense-prefix query blocks (i < pb) list every block.
 //
-// Rows of up to 4096 video key blocks take the scores from the tensor cores
+// Rows of up to 3072 video key blocks take the scores from the tensor cores
 // instead (select_tc_kernel, same phase 2):
-//  * one CTA per (R query blocks, head), R = 16 or 32; the MMA puts 128 key
+//  * one CTA per (R query blocks, head), R = 32 or 16; the MMA puts 128 key
 //    blocks on M (TMEM lanes) and the R query blocks on N, so the scores of
 //    key chunk c sit in TMEM columns [c R, c R + R) and stay there until
 //    every chunk is done;
@@ -29,8 +29,11 @@
 //    is within 2^-20 |x|); q.k = hi_q.hi_k + hi_q.lo_k + lo_q.hi_k, the
 //    dropped lo_q.lo_k being under 2^-20 |q_d k_d| as well;
 //  * TMA brings fp32 tiles of 32 dimensions (one 128-byte swizzle row) x 128
-//    pooled keys into a ring, four converter warps rewrite each tile in place
-//    as hi and write lo beside it, one thread issues the MMAs;
+//    pooled keys into a ring; four converter warps each take the rows of
+//    their TMEM lane quarter, split them in registers and store hi and lo to
+//    a TMEM tile (the MMA's A operand, so only the small query tile is read
+//    from shared memory: with A in shared memory the 4 KB it reads per MMA
+//    for only R columns bounded the score phase); one thread issues the MMAs;
 //  * then per batch of 8 query blocks the 8 warps copy the batch's scores
 //    from TMEM into shared memory (the staging space is free by then) and
 //    each warp selects one row.
@@ -359,22 +362,28 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const float* __restric
 
 // ---------------------------------------------------------- tensor-core scores
 
-constexpr int kTcThreads = 256;     // warp 0 TMA, 1 MMA + TMEM, 4-7 convert; all select
+// warp 0 TMA, 1 MMA + TMEM, 4-7 convert; all select (8 warps with two CTAs
+// per SM, 16 with one)
+constexpr int kTcMaxWarps = 16;
 constexpr uint32_t kKTile = 16384;  // 128 pooled keys x 32 fp32 (one swizzle row each)
-constexpr int kTcMaxStages = 6;
+constexpr int kTcMaxStages = 8;     // raw key tiles in flight
+constexpr int kTcAStages = 2;       // converted key tiles (TMEM, 64 columns each)
 
 struct TcCtl {
   uint64_t bfull, bconv, done;
-  uint64_t full[kTcMaxStages], conv[kTcMaxStages], empty[kTcMaxStages];
+  uint64_t full[kTcMaxStages], rempty[kTcMaxStages];
+  uint64_t conv[kTcAStages], aempty[kTcAStages];
   uint32_t tmem_base;
   int abort_flag;
-  uint32_t cbuf[kTcThreads / 32][64];   // per warp: the candidate keys of the top-k
+  uint32_t cbuf[kTcMaxWarps][64];   // per warp: the candidate keys of the top-k
 };
 
 struct TcCfg {
   int R;            // query blocks per CTA (MMA N)
-  int stages;       // key tiles in flight
-  uint32_t tcols;   // TMEM columns allocated (power of two >= chunks * R)
+  int warps;        // 8 (two CTAs per SM) or 16
+  int stages;       // raw key tiles in flight
+  uint32_t tcols;   // TMEM columns allocated (power of two)
+  uint32_t acol;    // first TMEM column of the converted key tiles
   int sstride;      // floats per score row of a phase-2 batch
   uint32_t off_ring, off_ctl;
   size_t smem;
@@ -386,13 +395,15 @@ __host__ __device__ constexpr uint32_t idesc_tf32_f32(uint32_t M, uint32_t N) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::tf32.  A (M=128 rows x K=8) sits in
+// TMEM with row i in lane i and one TF32 element per column (8 columns).
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -421,8 +432,8 @@ __device__ __forceinline__ void split_tf32(uint8_t* hi, uint8_t* lo, int n4, int
   }
 }
 
-template <int kPerLane, bool kThresh>
-__global__ void __launch_bounds__(kTcThreads, 2)
+template <int kPerLane, bool kThresh, int kW>
+__global__ void __launch_bounds__(kW * 32, kW == 8 ? 2 : 1)
     select_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k, int32_t* __restrict__ idx,
                      int32_t* __restrict__ cnt, int nb, int pb, int k_eff, int kcap,
@@ -447,8 +458,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     mbar_init(&ctl->done, 1);
     for (int st = 0; st < S; ++st) {
       mbar_init(&ctl->full[st], 1);
+      mbar_init(&ctl->rempty[st], 128);
+    }
+    for (int st = 0; st < kTcAStages; ++st) {
       mbar_init(&ctl->conv[st], 128);
-      mbar_init(&ctl->empty[st], 1);
+      mbar_init(&ctl->aempty[st], 1);
     }
     ctl->abort_flag = ((smem_u32(sm) & 1023u) != 0) ? 1 : 0;
     fence_barrier_init();
@@ -473,9 +487,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       int issued = 0;
       for (int it = 0; it < T; ++it) {
         const int st = it % S;
-        if (it >= S && !mbar_wait(&ctl->empty[st], ((it / S) - 1) & 1, wc)) break;
+        if (it >= S && !mbar_wait(&ctl->rempty[st], ((it / S) - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(&ctl->full[st], kKTile);
-        tma_load_3d(ring + st * 2 * kKTile, &tm_k, &ctl->full[st], 32 * (it & 3),
+        tma_load_3d(ring + st * kKTile, &tm_k, &ctl->full[st], 32 * (it & 3),
                     pb + kBlock * (it >> 2), bh);
         issued = it + 1;
       }
@@ -489,41 +503,63 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       const uint32_t idesc = idesc_tf32_f32(128, R);
       bool ok = mbar_wait(&ctl->bconv, 0, wc);
       for (int it = 0; it < T && ok; ++it) {
-        const int st = it % S, kb = it & 3;
-        if (!mbar_wait(&ctl->conv[st], (it / S) & 1, wc)) { ok = false; break; }
+        const int sa = it % kTcAStages, kb = it & 3;
+        if (!mbar_wait(&ctl->conv[sa], (it / kTcAStages) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + (it >> 2) * R;
-        const uint32_t ahi = smem_u32(ring + st * 2 * kKTile), alo = ahi + kKTile;
+        const uint32_t ahi = tmem + cfg.acol + 64 * sa, alo = ahi + 32;
         const uint32_t bh_ = smem_u32(bhi + kb * btile), bl_ = smem_u32(blo + kb * btile);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_tf32_ss(d, smem_desc_sw128(ahi + 32 * kk, 16, 1024),
-                      smem_desc_sw128(bh_ + 32 * kk, 16, 1024), idesc, (kb | kk) != 0);
+          mma_tf32_ts(d, ahi + 8 * kk, smem_desc_sw128(bh_ + 32 * kk, 16, 1024), idesc,
+                      (kb | kk) != 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_tf32_ss(d, smem_desc_sw128(ahi + 32 * kk, 16, 1024),
-                      smem_desc_sw128(bl_ + 32 * kk, 16, 1024), idesc, 1u);
+          mma_tf32_ts(d, ahi + 8 * kk, smem_desc_sw128(bl_ + 32 * kk, 16, 1024), idesc, 1u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_tf32_ss(d, smem_desc_sw128(alo + 32 * kk, 16, 1024),
-                      smem_desc_sw128(bh_ + 32 * kk, 16, 1024), idesc, 1u);
-        mma_commit(&ctl->empty[st]);
+          mma_tf32_ts(d, alo + 8 * kk, smem_desc_sw128(bh_ + 32 * kk, 16, 1024), idesc, 1u);
+        mma_commit(&ctl->aempty[sa]);
       }
       mma_commit(&ctl->done);
     }
-  } else if (run && warp >= 4) {
+  } else if (run && warp >= 4 && warp < 8) {
     const int t = tid - 128;
     bool ok = mbar_wait(&ctl->bfull, 0, wc);
     if (ok) split_tf32(bhi, blo, static_cast<int>(4 * btile / 16), t, 128);
     fence_proxy_async_smem();
     mbar_arrive(&ctl->bconv);
+    // key row r of each tile (TMEM lane r): its 32 dimensions, split, to TMEM
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lanes = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     for (int it = 0; it < T && ok; ++it) {
-      const int st = it % S;
+      const int st = it % S, sa = it % kTcAStages;
       if (!mbar_wait(&ctl->full[st], (it / S) & 1, wc)) { ok = false; break; }
-      split_tf32(ring + st * 2 * kKTile, ring + st * 2 * kKTile + kKTile,
-                 static_cast<int>(kKTile / 16), t, 128);
-      fence_proxy_async_smem();
-      mbar_arrive(&ctl->conv[st]);
+      if (it >= kTcAStages && !mbar_wait(&ctl->aempty[sa], ((it / kTcAStages) - 1) & 1, wc)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint8_t* row = ring + st * kKTile + r * 128;
+      uint32_t hi[32], lo[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 x = *reinterpret_cast<const float4*>(row + ((c ^ (r & 7)) << 4));
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t h = __float_as_uint(xs[u]) & 0xffffe000u;
+          hi[4 * c + u] = h;
+          lo[4 * c + u] = __float_as_uint(xs[u] - __uint_as_float(h));
+        }
+      }
+      mbar_arrive(&ctl->rempty[st]);   // the raw tile is in registers
+      const uint32_t a = tmem + lanes + cfg.acol + 64 * sa;
+      BSA_TMEM_ST_32(a, hi);
+      BSA_TMEM_ST_32(a + 32, lo);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&ctl->conv[sa]);
     }
   }
 
@@ -533,16 +569,20 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   tc_fence_after();
   if (ctl->abort_flag == 0) {
     float* sc = reinterpret_cast<float*>(sm);
-    const int g = warp & 3, half = warp >> 2;
-    for (int rb = 0; rb < R && i0 + rb < nb; rb += 8) {
-      for (int c = half; c < chunks; c += 2) {
-        uint32_t v[8];
-        tmem_ld8(tmem + (static_cast<uint32_t>(32 * g) << 16) + c * R + rb, v);
-        tmem_wait_ld();
+    const int g = warp & 3, part = warp >> 2;
+    for (int rb = 0; rb < R && i0 + rb < nb; rb += kW) {
+      for (int c = part; c < chunks; c += kW / 4) {
         const int key = kBlock * c + 32 * g + lane;
-        if (key < nbv) {
 #pragma unroll
-          for (int r = 0; r < 8; ++r) sc[r * cfg.sstride + key] = __uint_as_float(v[r]) * scale;
+        for (int r8 = 0; r8 < kW; r8 += 8) {
+          uint32_t v[8];
+          tmem_ld8(tmem + (static_cast<uint32_t>(32 * g) << 16) + c * R + rb + r8, v);
+          tmem_wait_ld();
+          if (key < nbv) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+              sc[(r8 + r) * cfg.sstride + key] = __uint_as_float(v[r]) * scale;
+          }
         }
       }
       __syncthreads();
@@ -558,31 +598,36 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   if (warp == 1) tmem_dealloc(tmem, cfg.tcols);
 }
 
-// Tensor-core configuration for nbv video key blocks, or R = 0 when a row of
-// scores does not fit (more than 4096 blocks).  `pair`: two CTAs per SM
-// (each within 256 TMEM columns and half the shared memory), so one CTA's
-// selection overlaps the other's score phase; otherwise one CTA per SM with
-// all 512 columns and a deeper ring.  R query blocks per CTA share every key
-// tile the CTA loads (32, else 16).  The score batch of phase 2 (8 rows)
-// reuses the staging space.
+// Tensor-core configuration for nbv video key blocks, or R = 0 when the
+// scores and two converted key tiles do not fit in TMEM (more than 3072
+// blocks).  `pair`: two CTAs per SM (each within 256 TMEM columns and half
+// the shared memory), so one CTA's selection overlaps the other's score
+// phase; otherwise one CTA per SM with all 512 columns and a deeper ring.  R
+// query blocks per CTA share every key tile the CTA loads (32, else 16).
+// The score batch of phase 2 (one row per warp) reuses the staging space.
 TcCfg tc_config(int nbv, bool pair) {
   TcCfg c{};
   const int chunks = (nbv + kBlock - 1) / kBlock;
   const int cols = pair ? 256 : 512;
-  if (nbv <= 0 || chunks * 16 > cols) return c;
-  c.R = chunks * 32 <= cols ? 32 : 16;
-  const uint32_t need = static_cast<uint32_t>(chunks * c.R);
+  const int acols = 64 * kTcAStages;
+  if (nbv <= 0 || ((chunks * 16 + 63) & ~63) + acols > cols) return c;
+  c.R = ((chunks * 32 + 63) & ~63) + acols <= cols ? 32 : 16;
+  c.acol = static_cast<uint32_t>((chunks * c.R + 63) & ~63);
+  const uint32_t need = c.acol + acols;
   c.tcols = 32;
   while (c.tcols < need) c.tcols <<= 1;
   c.sstride = (nbv + 3) & ~3;
-  const size_t batch = static_cast<size_t>(8) * c.sstride * 4;
   c.off_ring = static_cast<uint32_t>(c.R) * 1024;   // query tile: hi + lo, 4 slices each
   const size_t budget = pair ? 113 * 1024 : 224 * 1024;
   c.stages = kTcMaxStages;
-  while (c.stages > 2 && c.off_ring + c.stages * 2 * kKTile + sizeof(TcCtl) > budget) --c.stages;
-  c.off_ctl = c.off_ring + c.stages * 2 * kKTile;
+  while (c.stages > 2 && c.off_ring + c.stages * kKTile + sizeof(TcCtl) > budget) --c.stages;
+  c.off_ctl = c.off_ring + c.stages * kKTile;
   c.smem = c.off_ctl + sizeof(TcCtl);
-  if (batch > c.off_ctl || c.smem > budget) c.R = 0;
+  // one warp per row of a phase-2 batch: 16 where one CTA holds the SM and
+  // a batch of 16 score rows fits, else 8
+  const auto batch = [&](int w) { return static_cast<size_t>(w) * c.sstride * 4; };
+  c.warps = (!pair && c.R % 16 == 0 && batch(16) <= c.off_ctl) ? 16 : 8;
+  if (batch(c.warps) > c.off_ctl || c.smem > budget) c.R = 0;
   // one CTA per SM: ask for more than half of the SM's shared memory
   if (!pair && c.smem < 120 * 1024) c.smem = 120 * 1024;
   return c;
@@ -595,22 +640,29 @@ TcCfg tc_config(int nbv) {
   return p.R > 0 ? p : tc_config(nbv, false);
 }
 
-template <int kPerLane, bool kThresh = false>
-cudaError_t launch_select_tc(const Shape& s, const SelectMaps& maps, const TcCfg& cfg,
-                             int32_t* idx, int32_t* cnt, cudaStream_t st, float tau = 0.f) {
+template <int kPerLane, bool kThresh, int kW>
+cudaError_t launch_select_tc_w(const Shape& s, const SelectMaps& maps, const TcCfg& cfg,
+                               int32_t* idx, int32_t* cnt, cudaStream_t st, float tau) {
   static std::atomic<bool> attr_set[64];
   cudaError_t e = once_per_device(attr_set, [] {
-    return cudaFuncSetAttribute(select_tc_kernel<kPerLane, kThresh>,
+    return cudaFuncSetAttribute(select_tc_kernel<kPerLane, kThresh, kW>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 225 * 1024);
   });
   if (e != cudaSuccess) return e;
   const dim3 grid((s.nb + cfg.R - 1) / cfg.R, s.B * s.H);
   const float scale = 0.088388347648318440550f;
   const int kcap = kThresh ? s.nb : s.kcap;
-  select_tc_kernel<kPerLane, kThresh><<<grid, kTcThreads, cfg.smem, st>>>(
-      maps.q, maps.k, idx, cnt, s.nb, s.pb, s.k_eff, kcap, cfg, scale, tau,
-      s.dev_status);
+  select_tc_kernel<kPerLane, kThresh, kW><<<grid, kW * 32, cfg.smem, st>>>(
+      maps.q, maps.k, idx, cnt, s.nb, s.pb, s.k_eff, kcap, cfg, scale, tau, s.dev_status);
   return cudaGetLastError();
+}
+
+template <int kPerLane, bool kThresh = false>
+cudaError_t launch_select_tc(const Shape& s, const SelectMaps& maps, const TcCfg& cfg,
+                             int32_t* idx, int32_t* cnt, cudaStream_t st, float tau = 0.f) {
+  return cfg.warps == 16
+             ? launch_select_tc_w<kPerLane, kThresh, 16>(s, maps, cfg, idx, cnt, st, tau)
+             : launch_select_tc_w<kPerLane, kThresh, 8>(s, maps, cfg, idx, cnt, st, tau);
 }
 
 template <int kPerLane, bool kThresh = false>

@@ -1,10 +1,11 @@
 """GPU parity of the selection stage alone (bsa_select / bsa_select_threshold
 on pooled inputs given directly), at row lengths that take every kernel
 configuration:
-  * tensor-core scores, 32 query blocks per CTA (up to 2048 video blocks),
-    keys in registers (up to 1504 blocks) or in shared memory beyond;
-  * tensor-core scores, 16 query blocks per CTA (2049 to 4096 blocks);
-  * the SIMT kernel (more than 4096 blocks).
+  * tensor-core scores, two CTAs per SM (up to 512 video blocks) or one,
+    32 query blocks per CTA (up to 1984 blocks), keys in registers (up to
+    1504 blocks) or in shared memory beyond;
+  * tensor-core scores, 16 query blocks per CTA (1985 to 3072 blocks);
+  * the SIMT kernel (more than 3072 blocks).
 Selection is "each query block attends to its top-k key blocks"
 (h3-sparse-attn 0.1.0, opening description), or the threshold tau ("H3
 Sparse Attention", WAS node page, "The inputs that matter").  Pooled vectors
@@ -58,11 +59,11 @@ def _run(nbv, pb, kind, seed, top_k=None, tau=None):
 @pytest.mark.parametrize("nbv,top_k,pb,kind", [
     (295, 64, 0, "gauss"),      # 32 query blocks per CTA, 13 keys per lane
     (295, 64, 0, "ties"),
-    (1045, 64, 2, "gauss"),     # 2K-5s rows: 35 keys per lane, 512 TMEM columns
+    (1045, 64, 2, "gauss"),     # 2K-5s rows: 35 keys per lane, one CTA per SM
     (1400, 700, 0, "ties"),     # 47 keys per lane, half the row kept
     (1400, 1, 1, "gauss"),
     (1800, 64, 0, "gauss"),     # keys in shared memory
-    (3000, 64, 0, "gauss"),     # 16 query blocks per CTA
+    (3000, 64, 0, "gauss"),     # 16 query blocks per CTA, all 512 TMEM columns
     (3000, 5, 3, "ties"),
     (5000, 64, 0, "gauss"),     # SIMT scores
 ])
