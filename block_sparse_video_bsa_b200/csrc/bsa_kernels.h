@@ -122,6 +122,7 @@ struct ReblockPlan {
   int max_partials;       // chunk partials per head (largest level)
   int max_chunks[16];     // 2048-row chunks of the largest group, per level
   int max_pchunks[16];    // 512-position projection chunks of the largest group
+                          // (0: every group is projected in its Gram CTA)
 };
 ReblockPlan reblock_plan(const Shape& s);
 struct ReblockBuffers {

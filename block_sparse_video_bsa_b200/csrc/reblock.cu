@@ -24,7 +24,9 @@
 //   factor_kernel         Cholesky of M (fp64, one CTA per head); writes
 //                         R = L^T as bf16 hi + lo (R ~= hi + lo to ~16 bits).
 //   whiten_kernel         Y = Q R^T on tcgen05 (two MMAs per K step: hi, lo),
-//                         u = Y / |Y| stored bf16, one CTA per 128 tokens.
+//                         u = Y / |Y| stored bf16; persistent, one CTA per SM
+//                         over consecutive 128-token tiles (R loaded once per
+//                         head), TMA ring and two TMEM accumulators.
 //   per level (group j of level l found by descending the tree; the groups
 //   of a level are ranges of the working order `perm`):
 //   gram_kernel<group>    sum u u^T and sum u over a chunk of a group's
@@ -33,7 +35,9 @@
 //                         CTA, larger groups leave partials for group_kernel.
 //   group_kernel          fixed-order sum of a large group's partials, power
 //                         iteration.
-//   project_kernel        p = u . v per position -> order-preserving key.
+//   project_kernel        p = u . v per position -> order-preserving key
+//                         (groups of at most 3 tiles: in their Gram CTA,
+//                         whose ring still holds all their rows).
 //   split_kernel          radix select of the floor(b/2)*128-th key (four
 //                         8-bit passes over the group's keys, ties broken by
 //                         position), then a stable partition of perm.
@@ -82,25 +86,30 @@ __device__ __forceinline__ uint32_t swz(int r, int c16) {
   return static_cast<uint32_t>((c16 >> 3) * kHalf + r * 128 + ((((c16 & 7) ^ (r & 7))) << 4));
 }
 
-// 128 threads, thread i owns row i of G (in g[]); smem v[128], c[128] (mean),
-// red[4].  Writes the unit direction of kPowerIters iterations of
-// C = G - n c c^T from (1, ..., 1)/sqrt(128) to out[i].  A zero step keeps v.
-__device__ __forceinline__ void power_iterate(const float (&g)[128], float n, float* c, float* v,
+// 128 threads, thread i owns row i of G (in g[], overwritten by row i of the
+// centred scatter C = G - n c c^T); smem v[128] (16-byte aligned), c[128]
+// (mean), red[4].  Writes the unit direction of kPowerIters iterations of C
+// from (1, ..., 1)/sqrt(128) to out[i].  A zero step keeps v.
+__device__ __forceinline__ void power_iterate(float (&g)[128], float n, float* c, float* v,
                                               float* red, float* out) {
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const float nci = -n * c[i];
+#pragma unroll
+  for (int j = 0; j < 128; ++j) g[j] = fmaf(nci, c[j], g[j]);
   v[i] = 0.08838834764831845f;   // 1 / sqrt(128)
   __syncthreads();
   for (int it = 0; it < kPowerIters; ++it) {
-    // four independent partial sums per dot product (fixed order)
-    float cv4[4] = {0.f, 0.f, 0.f, 0.f}, w4[4] = {0.f, 0.f, 0.f, 0.f};
+    // four independent partial sums (fixed order), v read as broadcast float4s
+    float w4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll   // fully: g[] stays in registers
-    for (int j = 0; j < 128; ++j) {
-      cv4[j & 3] = fmaf(c[j], v[j], cv4[j & 3]);
-      w4[j & 3] = fmaf(g[j], v[j], w4[j & 3]);
+    for (int j4 = 0; j4 < 32; ++j4) {
+      const float4 vv = reinterpret_cast<const float4*>(v)[j4];
+      w4[0] = fmaf(g[4 * j4], vv.x, w4[0]);
+      w4[1] = fmaf(g[4 * j4 + 1], vv.y, w4[1]);
+      w4[2] = fmaf(g[4 * j4 + 2], vv.z, w4[2]);
+      w4[3] = fmaf(g[4 * j4 + 3], vv.w, w4[3]);
     }
-    const float cv = (cv4[0] + cv4[1]) + (cv4[2] + cv4[3]);
-    float w = (w4[0] + w4[1]) + (w4[2] + w4[3]);
-    w = fmaf(-n * c[i], cv, w);
+    const float w = (w4[0] + w4[1]) + (w4[2] + w4[3]);
     float s = w * w;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -122,16 +131,24 @@ struct GramArgs {
   float* part;              // [BH, slots * max_chunks, 128, 128]
   float* psum;              // [BH, slots * max_chunks, 128]  (group mode)
   float* vdir;              // [BH, slots, 128]                (group mode)
+  uint32_t* keys;           // [BH, nv] projection keys of small groups (group mode)
   int* dev_status;
 };
 
 constexpr int kStages = 3;   // Gram tiles in flight (cp.async ring)
+constexpr uint32_t kGramCols = 256;   // TMEM: Gram in columns 0-127, column sums 128-143
+// Groups of at most this many rows stay whole in the Gram CTA's ring, which
+// then also forms their projections (project_kernel skips them).
+constexpr int kGramProjRows = kStages * kBlock;
 
 struct GramSmem {
+  alignas(1024) uint16_t ones[16 * 64];   // bf16 1.0: B of the column-sum MMAs
   uint64_t done[kStages];
   uint32_t tmem_base;
   int abort_flag;
-  float c[128], v[128], red[4];
+  alignas(16) float c[128];
+  alignas(16) float v[128];
+  float red[4];
   int32_t rows[kChunkTok];   // group mode: u row of each position of the chunk
 };
 
@@ -164,12 +181,13 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
     fence_barrier_init();
   }
   if (tid < 32) {
-    tmem_alloc(&ctl->tmem_base, 128);
+    tmem_alloc(&ctl->tmem_base, kGramCols);
     tmem_relinquish();
   }
-  if constexpr (kGroup) {   // the chunk's rows of u, read once
+  if constexpr (kGroup) {   // the chunk's rows of u, read once; the ones tile
     for (int i = tid; i < p1 - p0; i += 128)
       ctl->rows[i] = __ldg(a.perm + bh * a.N + a.prefix + p0 + i) - a.prefix;
+    for (int e = tid; e < 16 * 64; e += 128) ctl->ones[e] = 0x3F80;   // bf16 1.0
   }
   tc_fence_before();
   __syncthreads();
@@ -177,6 +195,10 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
   const uint32_t tmem = ctl->tmem_base;
   const WaitCtx wc{&ctl->abort_flag, a.dev_status};
   const uint32_t idesc = idesc_bf16_f32_mn(128, 128);
+  // column sums: A = rows^T (MN-major) as for the Gram, B = ones (K-major, N = 16)
+  constexpr uint32_t idesc_cs = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+                                ((16u >> 3) << 17) | ((128u >> 4) << 24);
+  const uint32_t ones = smem_u32(ctl->ones);
 
   auto row_ptr = [&](int pos) -> const __nv_bfloat16* {
     if constexpr (kGroup) {
@@ -210,7 +232,6 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
   };
   issue_tile(0);
   issue_tile(1);
-  float colsum = 0.f;
   bool ok = true;
   for (int it = 0; it < ntile && ok; ++it) {
     // buffer (it + 2) % kStages last held tile it - 1: its MMAs must be done
@@ -227,21 +248,6 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
     fence_proxy_async_smem();
     __syncthreads();
     const uint8_t* buf = sm + (it % kStages) * kTile;
-    if constexpr (kGroup) {   // column tid of the tile's rows (rows past nrow are zero)
-      const int cc = tid >> 3, e = tid & 7;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll 4
-      for (int r = 0; r < kBlock; r += 4) {
-        s0 += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(buf + swz(r, cc) + 2 * e));
-        s1 += __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16*>(buf + swz(r + 1, cc) + 2 * e));
-        s2 += __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16*>(buf + swz(r + 2, cc) + 2 * e));
-        s3 += __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16*>(buf + swz(r + 3, cc) + 2 * e));
-      }
-      colsum += (s0 + s1) + (s2 + s3);
-    }
     if (tid == 0) {
       tc_fence_after();
       const uint32_t addr = smem_u32(buf);
@@ -249,6 +255,9 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
       for (int kk = 0; kk < 8; ++kk) {   // 16 rows per MMA
         const uint64_t d = smem_desc_sw128(addr + kk * 2048, kHalf, 1024);
         mma_bf16_ss(tmem, d, d, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+        if constexpr (kGroup)   // column sums: the same rows times a tile of ones
+          mma_bf16_ss(tmem + 128, d, smem_desc_sw128(ones + 32 * (kk & 3), 16, 1024), idesc_cs,
+                      (it > 0 || kk > 0) ? 1u : 0u);
       }
       mma_commit(&ctl->done[it % kStages]);
     }
@@ -267,6 +276,13 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
     BSA_TMEM_LD_32F(tmem + lane_base + 32, gr + 32);
     BSA_TMEM_LD_32F(tmem + lane_base + 64, gr + 64);
     BSA_TMEM_LD_32F(tmem + lane_base + 96, gr + 96);
+    float colsum = 0.f;
+    if constexpr (kGroup) {
+      uint32_t cs[8];
+      tmem_ld8(tmem + lane_base + 128, cs);
+      tmem_wait_ld();
+      colsum = __uint_as_float(cs[0]);
+    }
     tmem_wait_ld();
     const size_t pidx = static_cast<size_t>(bh) * a.slots * a.max_chunks +
                         static_cast<size_t>(slot) * a.max_chunks + chunk;
@@ -276,6 +292,31 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
       __syncthreads();
       power_iterate(gr, n, ctl->c, ctl->v, ctl->red,
                     a.vdir + (bh * a.slots + slot) * kDim);
+      if (g.count <= kGramProjRows) {
+        // p = u . v of every row (tile it sits in buffer it: ntile <= kStages),
+        // summed in project_kernel's order: eight products per 16-byte chunk,
+        // then the chunks pairwise as its lane butterfly does
+        for (int it = 0; it < ntile; ++it) {
+          const int pos = p0 + it * kBlock + tid;
+          if (pos >= p1) break;
+          const uint8_t* buf = sm + it * kTile;
+          float part[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4*>(buf + swz(tid, c));
+            const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&w);
+            float sc = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sc = fmaf(__bfloat162float(h[e]), ctl->v[8 * c + e], sc);
+            part[c] = sc;
+          }
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+            for (int c = 0; c < o; ++c) part[c] = part[c] + part[c + o];
+          a.keys[bh * a.nv + pos] = orderable_key(part[0]);
+        }
+      }
     } else {
       float4* dst = reinterpret_cast<float4*>(a.part + (pidx * 128 + tid) * 128);
 #pragma unroll
@@ -289,14 +330,16 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
   if (tid < 32) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, kGramCols);
   }
 }
 
 // Power iteration of a group larger than one chunk: fixed-order sum of its
 // chunk partials.
 __global__ void __launch_bounds__(128) group_kernel(const GramArgs a) {
-  __shared__ float c[128], v[128], red[4];
+  __shared__ alignas(16) float c[128];
+  __shared__ alignas(16) float v[128];
+  __shared__ float red[4];
   const int tid = threadIdx.x, slot = blockIdx.x;
   const size_t bh = blockIdx.y;
   const Range g = group_of(a.nv, a.level, slot);
@@ -308,15 +351,19 @@ __global__ void __launch_bounds__(128) group_kernel(const GramArgs a) {
   float s = 0.f;
   const size_t p0 = static_cast<size_t>(bh) * a.slots * a.max_chunks +
                     static_cast<size_t>(slot) * a.max_chunks;
+  // chunk by chunk in a fixed order; each chunk's row arrives as 32
+  // independent 16-byte loads issued together
   for (int ch = 0; ch < nch; ++ch) {
     const float4* src = reinterpret_cast<const float4*>(a.part + ((p0 + ch) * 128 + tid) * 128);
+    float4 x[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) x[q] = __ldg(src + q);
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
-      const float4 x = src[q];
-      gr[4 * q] += x.x;
-      gr[4 * q + 1] += x.y;
-      gr[4 * q + 2] += x.z;
-      gr[4 * q + 3] += x.w;
+      gr[4 * q] += x[q].x;
+      gr[4 * q + 1] += x[q].y;
+      gr[4 * q + 2] += x[q].z;
+      gr[4 * q + 3] += x[q].w;
     }
     s += a.psum[(p0 + ch) * 128 + tid];
   }
@@ -336,22 +383,11 @@ __global__ void __launch_bounds__(128) moment_reduce_kernel(const float* __restr
   M[(bh * 128 + i) * 128 + j] = s;
 }
 
-// dot of rows a and b of the shared matrix over k < n, four partial sums.
-__device__ __forceinline__ double row_dot(const double* a, const double* b, int n) {
-  double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-  int k = 0;
-  for (; k + 4 <= n; k += 4) {
-    s0 = fma(a[k], b[k], s0);
-    s1 = fma(a[k + 1], b[k + 1], s1);
-    s2 = fma(a[k + 2], b[k + 2], s2);
-    s3 = fma(a[k + 3], b[k + 3], s3);
-  }
-  for (; k < n; ++k) s0 = fma(a[k], b[k], s0);
-  return (s0 + s1) + (s2 + s3);
-}
-
 // Cholesky of the key second moment (fp64, in shared memory, lower triangle
-// in place) and R = L^T split into bf16 hi + lo.
+// in place) and R = L^T split into bf16 hi + lo.  Right-looking: for each
+// column j, the pivot's square root, the column below it scaled, then every
+// thread updates its own row of the trailing triangle (independent FMAs, so
+// a column costs one pass over a row rather than a chain of dot products).
 __global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ Mg,
                                                      __nv_bfloat16* __restrict__ r_hi,
                                                      __nv_bfloat16* __restrict__ r_lo) {
@@ -360,7 +396,14 @@ __global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ M
   const int tid = threadIdx.x;
   const size_t bh = blockIdx.x;
   constexpr int ld = 129;
-  for (int i = 0; i < 128; ++i) M[i * ld + tid] = Mg[(bh * 128 + i) * 128 + tid];
+  // the moment in batches of 16 independent loads per thread
+  for (int i0 = 0; i0 < 128; i0 += 16) {
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = __ldg(Mg + (bh * 128 + i0 + i) * 128 + tid);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) M[(i0 + i) * ld + tid] = x[i];
+  }
   __syncthreads();
   red[tid] = M[tid * ld + tid];
   __syncthreads();
@@ -373,15 +416,19 @@ __global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ M
   const double ridge = red[0];
   M[tid * ld + tid] += ridge;
   __syncthreads();
+  double* row = M + tid * ld;
   for (int j = 0; j < 128; ++j) {
-    if (tid == 0) {
-      const double s = M[j * ld + j] - row_dot(M + j * ld, M + j * ld, j);
-      M[j * ld + j] = sqrt(s > 0.0 ? s : 1e-300);
-    }
+    // every thread takes the pivot (one broadcast read) and scales its entry
+    const double s = M[j * ld + j];
+    const double d = sqrt(s > 0.0 ? s : 1e-300);
+    __syncthreads();   // all have read the pivot before its owner rewrites it
+    if (tid == j) row[j] = d;
+    if (tid > j) row[j] /= d;
     __syncthreads();
     if (tid > j) {
-      const double s = M[tid * ld + j] - row_dot(M + tid * ld, M + j * ld, j);
-      M[tid * ld + j] = s / M[j * ld + j];
+      const double lij = row[j];
+#pragma unroll 4
+      for (int k = j + 1; k <= tid; ++k) row[k] = fma(-lij, M[k * ld + j], row[k]);
     }
     __syncthreads();
   }
@@ -394,36 +441,53 @@ __global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ M
   }
 }
 
+constexpr int kWhThreads = 192;   // warps 0-3 epilogue (TMEM lane quarters), 4 TMA, 5 MMA
+constexpr int kWhStages = 3;      // Q tiles in flight
+constexpr uint32_t kWhOffQ = 2 * kTile;                       // after R hi, R lo
+constexpr uint32_t kWhOffCtl = kWhOffQ + kWhStages * kTile;
+
 struct WhitenSmem {
-  uint64_t full, done;
+  uint64_t rfull, rempty;                   // R (hi + lo) of the current head
+  uint64_t qfull[kWhStages], qempty[kWhStages];
+  uint64_t afull[2], aempty[2];             // two TMEM accumulators
+  uint64_t done;                            // every MMA of the CTA complete
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// u = Y / |Y|, Y = Q R^T (R ~= hi + lo), one CTA per 128 video tokens.
-__global__ void __launch_bounds__(128) whiten_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                     const __grid_constant__ CUtensorMap tm_hi,
-                                                     const __grid_constant__ CUtensorMap tm_lo,
-                                                     int prefix, int nv,
-                                                     __nv_bfloat16* __restrict__ u,
-                                                     int* dev_status) {
+// u = Y / |Y|, Y = Q R^T (R ~= hi + lo).  Persistent: CTA c takes the work
+// items [c * per, (c + 1) * per) of the (head, 128-token tile) sequence, so
+// it loads R once per head it meets; Q tiles stream through a 3-stage TMA
+// ring, and the epilogue of one tile (TMEM -> normalise -> store) overlaps
+// the MMAs of the next (two accumulators).
+__global__ void __launch_bounds__(kWhThreads, 1)
+    whiten_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_hi,
+                  const __grid_constant__ CUtensorMap tm_lo, int prefix, int nv, int ntile,
+                  int total, int per, __nv_bfloat16* __restrict__ u, int* dev_status) {
   extern __shared__ __align__(1024) uint8_t sm[];
-  WhitenSmem* ctl = reinterpret_cast<WhitenSmem*>(sm + 3 * kTile);
-  const int tid = threadIdx.x;
-  const int tile = blockIdx.x;
-  const int bh = blockIdx.y;
-  if ((smem_u32(sm) & 1023u) != 0) {
-    if (tid == 0 && dev_status) atomicExch(dev_status, kErrTimeout);
-    return;
-  }
+  WhitenSmem* ctl = reinterpret_cast<WhitenSmem*>(sm + kWhOffCtl);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int w0 = blockIdx.x * per, w1 = min(total, w0 + per);
+  if (w0 >= w1) return;
+  const int nw = w1 - w0;
   if (tid == 0) {
-    mbar_init(&ctl->full, 1);
+    mbar_init(&ctl->rfull, 1);
+    mbar_init(&ctl->rempty, 1);
+    for (int st = 0; st < kWhStages; ++st) {
+      mbar_init(&ctl->qfull[st], 1);
+      mbar_init(&ctl->qempty[st], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->afull[b], 1);
+      mbar_init(&ctl->aempty[b], 128);
+    }
     mbar_init(&ctl->done, 1);
-    ctl->abort_flag = 0;
+    ctl->abort_flag = ((smem_u32(sm) & 1023u) != 0) ? 1 : 0;
+    if (ctl->abort_flag && dev_status) atomicExch(dev_status, kErrTimeout);
     fence_barrier_init();
   }
-  if (tid < 32) {
-    tmem_alloc(&ctl->tmem_base, 128);
+  if (warp == 5) {
+    tmem_alloc(&ctl->tmem_base, 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -431,65 +495,114 @@ __global__ void __launch_bounds__(128) whiten_kernel(const __grid_constant__ CUt
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   const WaitCtx wc{&ctl->abort_flag, dev_status};
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&ctl->full, 3 * kTile);
-    const int row = prefix + tile * kBlock;
-    tma_load_3d(sm, &tm_q, &ctl->full, 0, row, bh);
-    tma_load_3d(sm + kHalf, &tm_q, &ctl->full, 64, row, bh);
-    tma_load_3d(sm + kTile, &tm_hi, &ctl->full, 0, 0, bh);
-    tma_load_3d(sm + kTile + kHalf, &tm_hi, &ctl->full, 64, 0, bh);
-    tma_load_3d(sm + 2 * kTile, &tm_lo, &ctl->full, 0, 0, bh);
-    tma_load_3d(sm + 2 * kTile + kHalf, &tm_lo, &ctl->full, 64, 0, bh);
-  }
-  bool ok = mbar_wait(&ctl->full, 0, wc);
-  if (tid == 0 && ok) {
-    tc_fence_after();
-    const uint32_t id = idesc_bf16_f32(128, 128, 0);
-    const uint32_t q = smem_u32(sm);
-    for (int part = 0; part < 2; ++part) {
-      const uint32_t rr = smem_u32(sm + (1 + part) * kTile);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-        mma_bf16_ss(tmem, smem_desc_sw128(q + off, 16, 1024), smem_desc_sw128(rr + off, 16, 1024),
-                    id, (part > 0 || kk > 0) ? 1u : 0u);
+  const bool run = ctl->abort_flag == 0;
+
+  if (run && warp == 4) {
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_hi);
+      prefetch_tensormap(&tm_lo);
+      int cur = -1, nr = 0, issued = 0;
+      bool ok = true;
+      for (int it = 0; it < nw && ok; ++it) {
+        const int w = w0 + it, bh = w / ntile, tile = w - bh * ntile;
+        if (bh != cur) {   // R of the new head, once the old head's MMAs are done
+          if (nr > 0 && !mbar_wait(&ctl->rempty, (nr - 1) & 1, wc)) { ok = false; break; }
+          mbar_arrive_expect_tx(&ctl->rfull, 2 * kTile);
+          tma_load_3d(sm, &tm_hi, &ctl->rfull, 0, 0, bh);
+          tma_load_3d(sm + kHalf, &tm_hi, &ctl->rfull, 64, 0, bh);
+          tma_load_3d(sm + kTile, &tm_lo, &ctl->rfull, 0, 0, bh);
+          tma_load_3d(sm + kTile + kHalf, &tm_lo, &ctl->rfull, 64, 0, bh);
+          ++nr;
+          cur = bh;
+        }
+        const int st = it % kWhStages;
+        if (it >= kWhStages && !mbar_wait(&ctl->qempty[st], ((it / kWhStages) - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        uint8_t* dst = sm + kWhOffQ + st * kTile;
+        const int row = prefix + tile * kBlock;
+        mbar_arrive_expect_tx(&ctl->qfull[st], kTile);
+        tma_load_3d(dst, &tm_q, &ctl->qfull[st], 0, row, bh);
+        tma_load_3d(dst + kHalf, &tm_q, &ctl->qfull[st], 64, row, bh);
+        issued = it + 1;
       }
+      // every issued load lands before the CTA moves on
+      if (nr > 0) mbar_wait(&ctl->rfull, (nr - 1) & 1, wc);
+      for (int k = (issued > kWhStages ? issued - kWhStages : 0); k < issued; ++k)
+        mbar_wait(&ctl->qfull[k % kWhStages], (k / kWhStages) & 1, wc);
     }
-    mma_commit(&ctl->done);
-  }
-  ok = __syncthreads_and(ok);
-  if (ok) ok = mbar_wait(&ctl->done, 0, wc);
-  ok = __syncthreads_and(ok);
-  tc_fence_after();
-  if (ok) {
-    const uint32_t lane_base = static_cast<uint32_t>((tid >> 5) * 32) << 16;
-    float y[128];
-    BSA_TMEM_LD_32F(tmem + lane_base, y);
-    BSA_TMEM_LD_32F(tmem + lane_base + 32, y + 32);
-    BSA_TMEM_LD_32F(tmem + lane_base + 64, y + 64);
-    BSA_TMEM_LD_32F(tmem + lane_base + 96, y + 96);
-    tmem_wait_ld();
-    const int t = tile * kBlock + tid;
-    if (t < nv) {
-      float ss = 0.f;
+  } else if (run && warp == 5) {
+    if (lane == 0) {
+      const uint32_t id = idesc_bf16_f32(128, 128, 0);
+      int cur = -1, nr = 0;
+      bool ok = true;
+      for (int it = 0; it < nw && ok; ++it) {
+        const int bh = (w0 + it) / ntile;
+        if (bh != cur) {
+          if (nr > 0) mma_commit(&ctl->rempty);   // the old head's MMAs release R
+          if (!mbar_wait(&ctl->rfull, nr & 1, wc)) { ok = false; break; }
+          ++nr;
+          cur = bh;
+        }
+        const int st = it % kWhStages, b = it & 1;
+        if (it >= 2 && !mbar_wait(&ctl->aempty[b], ((it >> 1) - 1) & 1, wc)) { ok = false; break; }
+        if (!mbar_wait(&ctl->qfull[st], (it / kWhStages) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t q = smem_u32(sm + kWhOffQ + st * kTile);
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t rr = smem_u32(sm + part * kTile);
 #pragma unroll
-      for (int j = 0; j < 128; ++j) ss = fmaf(y[j], y[j], ss);
-      const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(u + (static_cast<size_t>(bh) * nv + t) * kDim);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+            mma_bf16_ss(tmem + b * 128, smem_desc_sw128(q + off, 16, 1024),
+                        smem_desc_sw128(rr + off, 16, 1024), id, (part > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&ctl->qempty[st]);
+        mma_commit(&ctl->afull[b]);
+      }
+      // TMEM is freed only after every MMA issued here has finished
+      mma_commit(&ctl->done);
+      mbar_wait(&ctl->done, 0, wc);
+    }
+  } else if (run) {
+    // epilogue: thread tid = TMEM lane = token row of the tile
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    for (int it = 0; it < nw; ++it) {
+      const int w = w0 + it, bh = w / ntile, tile = w - bh * ntile, b = it & 1;
+      if (!mbar_wait(&ctl->afull[b], (it >> 1) & 1, wc)) break;
+      tc_fence_after();
+      float y[128];
+      BSA_TMEM_LD_32F(tmem + lane_base + b * 128, y);
+      BSA_TMEM_LD_32F(tmem + lane_base + b * 128 + 32, y + 32);
+      BSA_TMEM_LD_32F(tmem + lane_base + b * 128 + 64, y + 64);
+      BSA_TMEM_LD_32F(tmem + lane_base + b * 128 + 96, y + 96);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&ctl->aempty[b]);
+      const int t = tile * kBlock + tid;
+      if (t < nv) {
+        float ss = 0.f;
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
-        dst[q] = make_uint4(pack_bf16x2(y[8 * q] * inv, y[8 * q + 1] * inv),
-                            pack_bf16x2(y[8 * q + 2] * inv, y[8 * q + 3] * inv),
-                            pack_bf16x2(y[8 * q + 4] * inv, y[8 * q + 5] * inv),
-                            pack_bf16x2(y[8 * q + 6] * inv, y[8 * q + 7] * inv));
+        for (int j = 0; j < 128; ++j) ss = fmaf(y[j], y[j], ss);
+        const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(u + (static_cast<size_t>(bh) * nv + t) * kDim);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          dst[q] = make_uint4(pack_bf16x2(y[8 * q] * inv, y[8 * q + 1] * inv),
+                              pack_bf16x2(y[8 * q + 2] * inv, y[8 * q + 3] * inv),
+                              pack_bf16x2(y[8 * q + 4] * inv, y[8 * q + 5] * inv),
+                              pack_bf16x2(y[8 * q + 6] * inv, y[8 * q + 7] * inv));
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (tid < 32) {
-    __syncwarp();
+  if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -505,7 +618,7 @@ __global__ void __launch_bounds__(256) project_kernel(const __nv_bfloat16* __res
   const int slot = blockIdx.x / max_pchunks, chunk = blockIdx.x - slot * max_pchunks;
   const size_t bh = blockIdx.y;
   const Range g = group_of(nv, level, slot);
-  if (g.count <= kBlock) return;
+  if (g.count <= kGramProjRows) return;   // leaves; small groups are done in the Gram CTA
   const int p0 = g.start + chunk * kProjTok, p1 = min(p0 + kProjTok, g.start + g.count);
   if (p0 >= p1) return;
   if (tid < 128) v[tid] = vdir[(bh * slots + slot) * kDim + tid];
@@ -703,7 +816,9 @@ ReblockPlan reblock_plan(const Shape& s) {
   for (int l = 0; l < p.levels; ++l) {
     const int chunks = (largest + kChunkTok - 1) / kChunkTok;
     p.max_chunks[l] = chunks;
-    p.max_pchunks[l] = (largest + kProjTok - 1) / kProjTok;
+    // the rightmost group is the largest: none left for project_kernel when
+    // it fits in a Gram CTA's ring
+    p.max_pchunks[l] = largest > kGramProjRows ? (largest + kProjTok - 1) / kProjTok : 0;
     const long long parts = (chunks > 1) ? (static_cast<long long>(1) << l) * chunks : 1;
     if (parts > p.max_partials) p.max_partials = static_cast<int>(parts);
     const int m = ((largest + kBlock - 1) / kBlock / 2) * kBlock;
@@ -720,7 +835,7 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
   const int nv = plan.nv;
   // Gram kernels: two 32 KB tiles + control; factor: 128 x 129 doubles.
   const size_t gram_smem = kStages * kTile + sizeof(GramSmem) + 1024;
-  const size_t whiten_smem = 3 * kTile + sizeof(WhitenSmem) + 1024;
+  const size_t whiten_smem = kWhOffCtl + sizeof(WhitenSmem) + 1024;
   const size_t factor_smem = 128 * 129 * sizeof(double);
   static std::atomic<bool> attr[64];
   cudaError_t ea = once_per_device(attr, [&] {
@@ -749,6 +864,7 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
   ga.part = w.part;
   ga.psum = w.psum;
   ga.vdir = w.vdir;
+  ga.keys = w.keys;
   ga.dev_status = s.dev_status;
   // 1. key second moment (chunk partials), 2. factor, 3. whiten
   ga.X = static_cast<const __nv_bfloat16*>(K);
@@ -759,8 +875,17 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
   gram_kernel<false><<<dim3(plan.moment_chunks, BH), 128, gram_smem, st>>>(ga);
   moment_reduce_kernel<<<dim3(128, BH), 128, 0, st>>>(w.part, plan.moment_chunks, w.moment);
   factor_kernel<<<BH, 128, factor_smem, st>>>(w.moment, w.r_hi, w.r_lo);
-  whiten_kernel<<<dim3((nv + kBlock - 1) / kBlock, BH), 128, whiten_smem, st>>>(
-      maps.q, maps.r_hi, maps.r_lo, s.prefix, nv, w.u, s.dev_status);
+  {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int ntile = (nv + kBlock - 1) / kBlock;
+    const int total = BH * ntile;
+    const int ctas = total < sms ? total : sms;
+    const int per = (total + ctas - 1) / ctas;
+    whiten_kernel<<<(total + per - 1) / per, kWhThreads, whiten_smem, st>>>(
+        maps.q, maps.r_hi, maps.r_lo, s.prefix, nv, ntile, total, per, w.u, s.dev_status);
+  }
   (void)Q;
   // 4. levels
   ga.X = w.u;
@@ -775,8 +900,9 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
     ga.max_chunks = plan.max_chunks[l];
     gram_kernel<true><<<dim3(slots * plan.max_chunks[l], BH), 128, gram_smem, st>>>(ga);
     if (plan.max_chunks[l] > 1) group_kernel<<<dim3(slots, BH), 128, 0, st>>>(ga);
-    project_kernel<<<dim3(slots * plan.max_pchunks[l], BH), 256, 0, st>>>(
-        w.u, pa, w.vdir, s.N, s.prefix, nv, l, slots, plan.max_pchunks[l], w.keys);
+    if (plan.max_pchunks[l] > 0)
+      project_kernel<<<dim3(slots * plan.max_pchunks[l], BH), 256, 0, st>>>(
+          w.u, pa, w.vdir, s.N, s.prefix, nv, l, slots, plan.max_pchunks[l], w.keys);
     split_kernel<<<dim3(slots, BH), 512, 0, st>>>(w.keys, pa, pb, s.N, s.prefix, nv, l);
     int32_t* t = pa;
     pa = pb;

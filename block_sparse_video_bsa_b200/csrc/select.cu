@@ -407,14 +407,6 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// Eight consecutive TMEM columns of the warp's 32 lanes.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-                 "=r"(v[6]), "=r"(v[7])
-               : "r"(taddr));
-}
-
 // In place: each float of the n4 float4s at `hi` becomes its TF32 head (low 13
 // mantissa bits cleared); the remainder goes to the same place at `lo`.
 __device__ __forceinline__ void split_tf32(uint8_t* hi, uint8_t* lo, int n4, int t, int nt) {
