@@ -123,6 +123,7 @@ struct ReblockPlan {
   int max_chunks[16];     // 2048-row chunks of the largest group, per level
   int max_pchunks[16];    // 512-position projection chunks of the largest group
                           // (0: every group is projected in its Gram CTA)
+  int largest[16];        // tokens of the largest group, per level
 };
 ReblockPlan reblock_plan(const Shape& s);
 struct ReblockBuffers {

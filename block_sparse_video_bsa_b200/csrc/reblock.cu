@@ -21,7 +21,7 @@
 //                         swizzled layout, tcgen05.mma with A = B = rows^T
 //                         (MN-major), fp32 accumulator in TMEM; partials per
 //                         chunk, reduced in a fixed order by factor_kernel.
-//   factor_kernel         Cholesky of M (fp64, one CTA per head); writes
+//   factor_kernel         Cholesky of M (fp32, one CTA per head); writes
 //                         R = L^T as bf16 hi + lo (R ~= hi + lo to ~16 bits).
 //   whiten_kernel         Y = Q R^T on tcgen05 (two MMAs per K step: hi, lo),
 //                         u = Y / |Y| stored bf16; persistent, one CTA per SM
@@ -40,7 +40,9 @@
 //                         whose ring still holds all their rows).
 //   split_kernel          radix select of the floor(b/2)*128-th key (four
 //                         8-bit passes over the group's keys, ties broken by
-//                         position), then a stable partition of perm.
+//                         position), then a stable partition of perm
+//                         (split_small_kernel: one warp per group where no
+//                         group of the level exceeds 1024 keys).
 //   permute / unpermute   row gathers of Q, K, V into the new layout and the
 //                         scatter of O and lse back.
 // Every wait is bounded (globaltimer); on expiry the CTA records
@@ -383,16 +385,22 @@ __global__ void __launch_bounds__(128) moment_reduce_kernel(const float* __restr
   M[(bh * 128 + i) * 128 + j] = s;
 }
 
-// Cholesky of the key second moment (fp64, in shared memory, lower triangle
+// Cholesky of the key second moment (fp32, in shared memory, lower triangle
 // in place) and R = L^T split into bf16 hi + lo.  Right-looking: for each
 // column j, the pivot's square root, the column below it scaled, then every
-// thread updates its own row of the trailing triangle (independent FMAs, so
-// a column costs one pass over a row rather than a chain of dot products).
+// thread updates its own row of the trailing triangle (independent FMAs).
+// fp32 rather than fp64: FP64 runs at about one FMA per SM clock on this
+// part (an fp64 version took 0.26 ms for these 350k FMAs per head), and M
+// itself arrives as fp32 sums, so a backward-stable fp32 factor (L L^T =
+// M + E, |E| <~ 128 * 2^-24 |L| |L^T|) adds an error of the order already in
+// M, far below the bf16 rounding of the whitened vectors.  The trace (for
+// the ridge) is summed in fp64.
 __global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ Mg,
                                                      __nv_bfloat16* __restrict__ r_hi,
                                                      __nv_bfloat16* __restrict__ r_lo) {
-  extern __shared__ double M[];   // [128][129]
+  extern __shared__ float M[];     // [128][129]
   __shared__ double red[128];
+  __shared__ float col[128];       // the scaled column j (a separate array: no aliasing)
   const int tid = threadIdx.x;
   const size_t bh = blockIdx.x;
   constexpr int ld = 129;
@@ -413,28 +421,40 @@ __global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ M
     red[0] = 1e-6 * tr / 128.0;
   }
   __syncthreads();
-  const double ridge = red[0];
+  const float ridge = static_cast<float>(red[0]);
   M[tid * ld + tid] += ridge;
   __syncthreads();
-  double* row = M + tid * ld;
+  float* row = M + tid * ld;
   for (int j = 0; j < 128; ++j) {
     // every thread takes the pivot (one broadcast read) and scales its entry
-    const double s = M[j * ld + j];
-    const double d = sqrt(s > 0.0 ? s : 1e-300);
-    __syncthreads();   // all have read the pivot before its owner rewrites it
-    if (tid == j) row[j] = d;
-    if (tid > j) row[j] /= d;
-    __syncthreads();
+    const float s = M[j * ld + j];
+    const float d = sqrtf(s > 0.f ? s : 1e-30f);
+    float lij = 0.f;
     if (tid > j) {
-      const double lij = row[j];
-#pragma unroll 4
-      for (int k = j + 1; k <= tid; ++k) row[k] = fma(-lij, M[k * ld + j], row[k]);
+      lij = row[j] / d;
+      row[j] = lij;
+      col[tid] = lij;
+    }
+    __syncthreads();   // pivot read by all, column j in col[]
+    if (tid == j) row[j] = d;
+    if (tid > j) {
+      // four entries per step: all loads issued before the FMAs and stores
+      int k = j + 1;
+      for (; k + 3 <= tid; k += 4) {
+        const float c0 = col[k], c1 = col[k + 1], c2 = col[k + 2], c3 = col[k + 3];
+        const float r0 = row[k], r1 = row[k + 1], r2 = row[k + 2], r3 = row[k + 3];
+        row[k] = fmaf(-lij, c0, r0);
+        row[k + 1] = fmaf(-lij, c1, r1);
+        row[k + 2] = fmaf(-lij, c2, r2);
+        row[k + 3] = fmaf(-lij, c3, r3);
+      }
+      for (; k <= tid; ++k) row[k] = fmaf(-lij, col[k], row[k]);
     }
     __syncthreads();
   }
   // R = L^T: R[i][j] = L[j][i] for j >= i; thread tid writes column j = tid
   for (int i = 0; i < 128; ++i) {
-    const float r = tid >= i ? static_cast<float>(M[tid * ld + i]) : 0.f;
+    const float r = tid >= i ? M[tid * ld + i] : 0.f;
     const __nv_bfloat16 hi = __float2bfloat16_rn(r);
     r_hi[(bh * 128 + i) * 128 + tid] = hi;
     r_lo[(bh * 128 + i) * 128 + tid] = __float2bfloat16_rn(r - __bfloat162float(hi));
@@ -760,6 +780,66 @@ __global__ void __launch_bounds__(512) split_kernel(const uint32_t* __restrict__
   }
 }
 
+// The same split for a level whose groups hold at most 1024 keys: one warp
+// per group, the keys in registers (key of position lane + 32 e in slot e).
+// The m-th smallest key T is the (count - m + 1)-th largest, found by a
+// bitwise binary search with warp-wide counts; keys below T go left with the
+// lowest-position keys equal to T, each side keeping position order.
+constexpr int kSplitSmall = 1024;
+__global__ void __launch_bounds__(256) split_small_kernel(const uint32_t* __restrict__ keys,
+                                                          const int32_t* __restrict__ perm_in,
+                                                          int32_t* __restrict__ perm_out, int N,
+                                                          int prefix, int nv, int level,
+                                                          int slots) {
+  const int lane = threadIdx.x & 31;
+  const int slot = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const size_t bh = blockIdx.y;
+  if (slot >= slots) return;
+  const Range g = group_of(nv, level, slot);
+  if (g.count <= kBlock || g.count > kSplitSmall) return;
+  const int m = ((g.count + kBlock - 1) / kBlock / 2) * kBlock;
+  const uint32_t* k = keys + bh * nv + g.start;
+  uint32_t x[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const int i = lane + 32 * e;
+    x[e] = i < g.count ? __ldg(k + i) : 0u;
+  }
+  // T: the largest value with #{key >= T} >= count - m + 1 (padding is 0 and
+  // never counts: every candidate has a bit set)
+  const int kth = g.count - m + 1;
+  uint32_t T = 0;
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t cand = T | (1u << b);
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) c += (lane + 32 * e < g.count && x[e] >= cand) ? 1 : 0;
+    if (__reduce_add_sync(0xffffffffu, c) >= kth) T = cand;
+  }
+  int lt = 0;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) lt += (lane + 32 * e < g.count && x[e] < T) ? 1 : 0;
+  const int need_eq = m - __reduce_add_sync(0xffffffffu, lt);
+  const int32_t* pin = perm_in + bh * N + prefix + g.start;
+  int32_t* pout = perm_out + bh * N + prefix + g.start;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int left_run = 0, eq_run = 0;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    if (32 * e >= g.count) break;
+    const int i = lane + 32 * e;
+    const bool valid = i < g.count;
+    const bool is_eq = valid && x[e] == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+    const bool left = valid && (x[e] < T || (is_eq && eq_run + __popc(eqm & lt_mask) < need_eq));
+    const uint32_t lm = __ballot_sync(0xffffffffu, left);
+    const int l_before = left_run + __popc(lm & lt_mask);
+    if (valid) pout[left ? l_before : m + (i - l_before)] = __ldg(pin + i);
+    left_run += __popc(lm);
+    eq_run += __popc(eqm);
+  }
+}
+
 __global__ void init_perm_kernel(int32_t* __restrict__ perm, int N) {
   const size_t bh = blockIdx.y;
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < N; t += gridDim.x * blockDim.x)
@@ -819,6 +899,7 @@ ReblockPlan reblock_plan(const Shape& s) {
     // the rightmost group is the largest: none left for project_kernel when
     // it fits in a Gram CTA's ring
     p.max_pchunks[l] = largest > kGramProjRows ? (largest + kProjTok - 1) / kProjTok : 0;
+    p.largest[l] = largest;
     const long long parts = (chunks > 1) ? (static_cast<long long>(1) << l) * chunks : 1;
     if (parts > p.max_partials) p.max_partials = static_cast<int>(parts);
     const int m = ((largest + kBlock - 1) / kBlock / 2) * kBlock;
@@ -833,10 +914,10 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
                            cudaStream_t st) {
   const int BH = s.B * s.H;
   const int nv = plan.nv;
-  // Gram kernels: two 32 KB tiles + control; factor: 128 x 129 doubles.
+  // Gram kernels: three 32 KB tiles + control; factor: 128 x 129 floats.
   const size_t gram_smem = kStages * kTile + sizeof(GramSmem) + 1024;
   const size_t whiten_smem = kWhOffCtl + sizeof(WhitenSmem) + 1024;
-  const size_t factor_smem = 128 * 129 * sizeof(double);
+  const size_t factor_smem = 128 * 129 * sizeof(float);
   static std::atomic<bool> attr[64];
   cudaError_t ea = once_per_device(attr, [&] {
     cudaError_t e;
@@ -903,7 +984,11 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
     if (plan.max_pchunks[l] > 0)
       project_kernel<<<dim3(slots * plan.max_pchunks[l], BH), 256, 0, st>>>(
           w.u, pa, w.vdir, s.N, s.prefix, nv, l, slots, plan.max_pchunks[l], w.keys);
-    split_kernel<<<dim3(slots, BH), 512, 0, st>>>(w.keys, pa, pb, s.N, s.prefix, nv, l);
+    if (plan.largest[l] <= kSplitSmall)
+      split_small_kernel<<<dim3((slots + 7) / 8, BH), 256, 0, st>>>(w.keys, pa, pb, s.N,
+                                                                    s.prefix, nv, l, slots);
+    else
+      split_kernel<<<dim3(slots, BH), 512, 0, st>>>(w.keys, pa, pb, s.N, s.prefix, nv, l);
     int32_t* t = pa;
     pa = pb;
     pb = t;
