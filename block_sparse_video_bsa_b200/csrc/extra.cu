@@ -66,8 +66,8 @@ struct SelCtl {
   int abort_flag;
   int skip;
   // per selection warp: the 32 scores of a column group of every lane, [column][lane],
-  // read back by the lanes' appends
-  float xs[4][32][32];
+  // read back by the lanes' appends; the compaction's 64-key scratch in between
+  alignas(16) float xs[4][32][32];
 };
 static_assert(kOffSelCtl + sizeof(SelCtl) <= 227 * 1024, "shared memory budget");
 
@@ -107,8 +107,24 @@ __device__ __forceinline__ float key_score(unsigned long long key) {
 // half of the keys, then, when several keys share that score, on the token
 // half among them (a single one is found by a minimum).  Requires
 // 1 <= target <= count <= 32 * kSlots.
+// Exclusive prefix sum of v over the lanes of the warp.
+__device__ __forceinline__ int lane_prefix(int v, int lane) {
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x - v;
+}
+
+// The search over the score halves counts all keys only until the range
+// [th, th + 2^b) known to hold the target-th largest score holds at most 64
+// keys; those go to `scratch` (64 keys, the warp's own), two per lane, and the
+// search (and the token-half search among equal scores) finishes on them.
 template <int kSlots>
-__device__ unsigned long long compact_keys(unsigned long long* buf, int count, int target) {
+__device__ unsigned long long compact_keys(unsigned long long* buf, int count, int target,
+                                           unsigned long long* scratch) {
   const int lane = threadIdx.x & 31;
   __syncwarp();   // the owner's appends are visible to every lane
   uint32_t hi[kSlots], lo[kSlots];
@@ -123,38 +139,91 @@ __device__ unsigned long long compact_keys(unsigned long long* buf, int count, i
   // largest T_hi with #{hi >= T_hi} >= target (empty slots have hi = 0 and
   // every real key has hi > 0)
   uint32_t th = 0;
-  for (int b = 31; b >= 0; --b) {
+  int above = 0, at_least = count;   // keys with hi at or above the range's top / >= th
+  int b = 31;
+  for (; b >= 0; --b) {
     const uint32_t cand = th | (1u << b);
     int c4[4] = {0, 0, 0, 0};   // independent partial counts
 #pragma unroll
     for (int k = 0; k < kSlots; ++k) c4[k & 3] += hi[k] >= cand ? 1 : 0;
-    const int c = (c4[0] + c4[1]) + (c4[2] + c4[3]);
-    if (static_cast<int>(__reduce_add_sync(0xffffffffu, c)) >= target) th = cand;
-  }
-  int gt = 0, eq = 0;
-  uint32_t eq_min = 0xffffffffu;
-#pragma unroll
-  for (int k = 0; k < kSlots; ++k) {
-    gt += hi[k] > th ? 1 : 0;
-    if (hi[k] == th) {
-      ++eq;
-      eq_min = min(eq_min, lo[k]);
+    const int c =
+        static_cast<int>(__reduce_add_sync(0xffffffffu, (c4[0] + c4[1]) + (c4[2] + c4[3])));
+    if (c >= target) {
+      th = cand;
+      at_least = c;
+    } else {
+      above = c;
     }
+    if (at_least - above <= 64) break;
   }
-  gt = static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
-  eq = static_cast<int>(__reduce_add_sync(0xffffffffu, eq));
-  const int need = target - gt;   // 1 <= need <= eq
+  int gt, eq;
   uint32_t tl;
-  if (need == eq) {
-    tl = __reduce_min_sync(0xffffffffu, eq_min);
-  } else {   // several keys share the score: the need-th largest token half among them
-    tl = 0;
-    for (int b = 31; b >= 0; --b) {
-      const uint32_t cand = tl | (1u << b);
-      int c = 0;
+  if (b > 0) {
+    // the range's keys (at most 64) to the scratch, two per lane
+    const uint32_t width = 1u << b;
+    int own = 0;
 #pragma unroll
-      for (int k = 0; k < kSlots; ++k) c += (hi[k] == th && lo[k] >= cand) ? 1 : 0;
-      if (static_cast<int>(__reduce_add_sync(0xffffffffu, c)) >= need) tl = cand;
+    for (int k = 0; k < kSlots; ++k) own += (hi[k] != 0u && hi[k] - th < width) ? 1 : 0;
+    int pos = lane_prefix(own, lane);
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k)
+      if (hi[k] != 0u && hi[k] - th < width)
+        scratch[pos++] = (static_cast<unsigned long long>(hi[k]) << 32) | lo[k];
+    __syncwarp();
+    const int nc = at_least - above;
+    const unsigned long long e0 = lane < nc ? scratch[lane] : 0ull;
+    const unsigned long long e1 = lane + 32 < nc ? scratch[lane + 32] : 0ull;
+    __syncwarp();
+    const uint32_t h0 = static_cast<uint32_t>(e0 >> 32), h1 = static_cast<uint32_t>(e1 >> 32);
+    const uint32_t l0 = static_cast<uint32_t>(e0), l1 = static_cast<uint32_t>(e1);
+    // every candidate lies below the keys counted in `above`
+    for (--b; b >= 0; --b) {
+      const uint32_t cand = th | (1u << b);
+      const int c = above + static_cast<int>(__reduce_add_sync(
+                                0xffffffffu, (h0 >= cand ? 1 : 0) + (h1 >= cand ? 1 : 0)));
+      if (c >= target) th = cand;
+    }
+    gt = above + static_cast<int>(
+                     __reduce_add_sync(0xffffffffu, (h0 > th ? 1 : 0) + (h1 > th ? 1 : 0)));
+    const bool q0 = lane < nc && h0 == th, q1 = lane + 32 < nc && h1 == th;
+    eq = static_cast<int>(__reduce_add_sync(0xffffffffu, (q0 ? 1 : 0) + (q1 ? 1 : 0)));
+    const int need = target - gt;   // 1 <= need <= eq
+    if (need == eq) {
+      tl = __reduce_min_sync(0xffffffffu, min(q0 ? l0 : 0xffffffffu, q1 ? l1 : 0xffffffffu));
+    } else {   // several keys share the score: the need-th largest token half among them
+      tl = 0;
+      for (int bb = 31; bb >= 0; --bb) {
+        const uint32_t cand = tl | (1u << bb);
+        const int c = static_cast<int>(__reduce_add_sync(
+            0xffffffffu, ((q0 && l0 >= cand) ? 1 : 0) + ((q1 && l1 >= cand) ? 1 : 0)));
+        if (c >= need) tl = cand;
+      }
+    }
+  } else {
+    int g = 0, q = 0;
+    uint32_t eq_min = 0xffffffffu;
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k) {
+      g += hi[k] > th ? 1 : 0;
+      if (hi[k] == th) {
+        ++q;
+        eq_min = min(eq_min, lo[k]);
+      }
+    }
+    gt = static_cast<int>(__reduce_add_sync(0xffffffffu, g));
+    eq = static_cast<int>(__reduce_add_sync(0xffffffffu, q));
+    const int need = target - gt;   // 1 <= need <= eq
+    if (need == eq) {
+      tl = __reduce_min_sync(0xffffffffu, eq_min);
+    } else {   // several keys share the score: the need-th largest token half among them
+      tl = 0;
+      for (int bb = 31; bb >= 0; --bb) {
+        const uint32_t cand = tl | (1u << bb);
+        int c = 0;
+#pragma unroll
+        for (int k = 0; k < kSlots; ++k) c += (hi[k] == th && lo[k] >= cand) ? 1 : 0;
+        if (static_cast<int>(__reduce_add_sync(0xffffffffu, c)) >= need) tl = cand;
+      }
     }
   }
   const unsigned long long T = (static_cast<unsigned long long>(th) << 32) | tl;
@@ -371,7 +440,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         unsigned long long* rb = reinterpret_cast<unsigned long long*>(
             __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(buf), L));
         const int count = __shfl_sync(0xffffffffu, bcnt, L);
-        const unsigned long long t = compact_keys<kSlots>(rb, count, a.n_extra);
+        const unsigned long long t = compact_keys<kSlots>(
+            rb, count, a.n_extra, reinterpret_cast<unsigned long long*>(&xsw[0][0]));
         if (lane == L) {
           bcnt = a.n_extra;
           thr = t;
@@ -408,11 +478,11 @@ __global__ void __launch_bounds__(kFinThreads) extra_finish_kernel(const SelArgs
   const int bh = rowv / a.nbv, i = a.pb + rowv % a.nbv;
   unsigned long long* rb = a.cand + static_cast<size_t>(rowv) * kCap;
   int count = max(0, min(__ldg(a.bcnt + rowv), kCap));
+  uint32_t* tok = sbuf[warp];
   if (count > a.n_extra) {
-    compact_keys<kCap / 32>(rb, count, a.n_extra);
+    compact_keys<kCap / 32>(rb, count, a.n_extra, reinterpret_cast<unsigned long long*>(tok));
     count = a.n_extra;
   }
-  uint32_t* tok = sbuf[warp];
   for (int p = lane; p < count; p += 32) tok[p] = ~static_cast<uint32_t>(rb[p]);
   for (int p = count + lane; p < ((count + 3) & ~3); p += 32) tok[p] = 0xffffffffu;
   __syncwarp();
@@ -665,7 +735,10 @@ cudaError_t launch_select_extra_t(const Shape& s, const CUtensorMap& tm_k, const
 
 }  // namespace
 
-int extra_cand_cap(int n_extra) { return n_extra <= 256 ? 1280 : 2048; }
+// Candidate keys per query block: 768 up to 256 extra tokens (measured at
+// 256 on 768p-5s / 2K-5s: 4.00 / 17.1 ms against 4.20 / 18.4 with 1280 and
+// 4.57 / 18.3 with 512), 2048 above.
+int extra_cand_cap(int n_extra) { return n_extra <= 256 ? 768 : 2048; }
 
 size_t select_extra_scratch_bytes(const Shape& s, int n_extra) {
   if (n_extra <= 0) return 0;
@@ -699,8 +772,8 @@ cudaError_t launch_select_extra(const Shape& s, int n_extra, const CUtensorMap& 
   a.nbv = s.nbv;
   a.kcap = kcap;
   a.n_extra = n_extra;
-  return extra_cand_cap(n_extra) == 1280 ? launch_select_extra_t<1280>(s, tm_k, a, st)
-                                         : launch_select_extra_t<2048>(s, tm_k, a, st);
+  return extra_cand_cap(n_extra) == 768 ? launch_select_extra_t<768>(s, tm_k, a, st)
+                                        : launch_select_extra_t<2048>(s, tm_k, a, st);
 }
 
 cudaError_t launch_extra_summaries(const Shape& s, int n_extra, const void* K, const void* V,
