@@ -9,7 +9,8 @@ One step = one whole attention call (pool -> summarize -> select -> attend,
 all through the C ABI) over one batch of synthetic bf16 input of the 768p-5s
 H3 shape (B=1, H=56, N=37,740, d=128, top_k=64, anchor-weighted summaries).
 ``--reblock`` times the adaptive-reblocking option: the reblocked layout
-(bsa_reblock), the row gathers into it, the four stages on it and the scatter
+(bsa_reblock), the four stages on it (pool and summarize gathering the rows
+through the permutation) and the scatter
 of O back, every step.
 ``--precision fp8`` times the FP8 (e4m3) option instead: the same stages plus
 the quantisation of the attention operands, then the e4m3 attention kernel;
@@ -94,8 +95,9 @@ def parse_args():
 def reblock_launches(N: int, prefix: int) -> int:
     """Kernels bsa_reblock launches (its tree shape depends on N - prefix only):
     init + key moment (Gram, reduction) + factor + whiten, then per level a
-    Gram, a projection and a split, plus a partial-sum pass on levels whose
-    largest group spans more than one 2048-row chunk."""
+    Gram and a split, a projection on levels whose largest group exceeds 384
+    rows (smaller groups are projected in their Gram CTA), and a partial-sum
+    pass on levels whose largest group spans more than one 2048-row chunk."""
     nv = N - prefix
     levels = 0
     while (128 << levels) < nv:
@@ -104,7 +106,7 @@ def reblock_launches(N: int, prefix: int) -> int:
         return 1
     n, largest = 5, nv
     for _ in range(levels):
-        n += 3 + (1 if largest > 2048 else 0)
+        n += 2 + (1 if largest > 384 else 0) + (1 if largest > 2048 else 0)
         largest -= ((largest + 127) // 128 // 2) * 128
     return n
 
@@ -503,7 +505,7 @@ def main():
         Qa, Ka, Va, Oa = (torch.empty_like(Q) for _ in range(4))
     else:
         Qa, Ka, Va, Oa = Q, K, V, O
-    names = (["reblock", "permute"] if rbl else []) + ["pool", "summarize", "select"] + \
+    names = (["reblock"] if rbl else []) + ["pool", "summarize", "select"] + \
         (["quantize"] if fp8 else []) + (["select_extra", "extra_summaries"] if xtr else []) + \
         ["attend"] + (["unpermute"] if rbl else []) + (["gather"] if gather else [])
     nev = len(names) + 1
@@ -515,14 +517,17 @@ def main():
             if ev:
                 next(marks).record(stream)
         mark()
-        if rbl:
+        if rbl:   # the reblocked layout: pool and summarize gather Q, K, V through perm
             bsa.bsa_reblock(p, Q, K, perm, rb_ws, stream)
             mark()
-            bsa.bsa_permute(p, Q, K, V, perm, Qa, Ka, Va, stream)
-            mark()
-        bsa.bsa_pool(p, Qa, buf["qpool"], buf["anchor"], stream)
+            bsa.bsa_pool_permuted(p, Q, perm, Qa, buf["qpool"], buf["anchor"], stream)
+        else:
+            bsa.bsa_pool(p, Qa, buf["qpool"], buf["anchor"], stream)
         mark()
-        if xtr:
+        if rbl:
+            bsa.bsa_summarize_permuted(p, K, V, perm, Ka, Va, buf["anchor"], buf["kpool"],
+                                       buf["ksum"], buf["vsum"], buf["bias"], stream)
+        elif xtr:
             bsa.bsa_summarize_stats(p, K, V, buf["anchor"], buf["kpool"], buf["ksum"],
                                     buf["vsum"], buf["bias"], buf["kstat"], buf["vstat"],
                                     buf["lse_blk"], stream)
@@ -696,6 +701,8 @@ def main():
     pool_bytes = stage_bytes(B, H, N, nb, bsa.bsa_select_capacity(p))
     if xtr:   # summarize also writes the fp32 statistics of the side summaries
         pool_bytes += B * H * nb * (512 + 512 + 4)
+    if rbl:   # pool and summarize also write the permuted Q, K, V
+        pool_bytes += 3 * B * H * N * 256
     pool_gbs = pool_bytes / ((stage_ms[names.index("pool")] + stage_ms[names.index("summarize")])
                              / 1e3) / 1e9
 
@@ -749,7 +756,7 @@ def main():
             "e2e": e2e,
             "gpu_launches": ((11 if fp8 else (6 if thr else
                                               (5 + (2 if args.extra_tokens else 0) if xtr else 5)))
-                             + (reblock_launches(N, prefix) + 2 if rbl else 0)) * args.steps,
+                             + (reblock_launches(N, prefix) + 1 if rbl else 0)) * args.steps,
             "clocks": clock_info,
             "context": {"pages_rtx_pro_6000_sparse_ms": 30.7 if cfg["N"] == 37_740 else None},
         }

@@ -70,6 +70,9 @@ _SIGS = {
     "bsa_reblock_workspace_bytes": (ctypes.c_size_t, [_P]),
     "bsa_reblock": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "bsa_permute": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_pool_permuted": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "bsa_summarize_permuted": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                              _vp, _vp]),
     "bsa_unpermute": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp]),
     "bsa_forward_reblock_workspace_bytes": (ctypes.c_size_t, [_P]),
     "bsa_forward_reblock": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
@@ -249,6 +252,18 @@ def bsa_reblock(p, Q, K, perm, workspace, stream=None):
     _check(lib().bsa_reblock(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(perm), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)),
            "bsa_reblock")
+
+
+def bsa_pool_permuted(p, Q, perm, Qp, qpool, anchor, stream=None):
+    _check(lib().bsa_pool_permuted(ctypes.byref(p), _ptr(Q), _ptr(perm), _ptr(Qp), _ptr(qpool),
+                                   _ptr(anchor), _stream(stream)), "bsa_pool_permuted")
+
+
+def bsa_summarize_permuted(p, K, V, perm, Kp, Vp, anchor, kpool, ksum, vsum, bias, stream=None):
+    _check(lib().bsa_summarize_permuted(ctypes.byref(p), _ptr(K), _ptr(V), _ptr(perm), _ptr(Kp),
+                                        _ptr(Vp), _ptr(anchor), _ptr(kpool), _ptr(ksum),
+                                        _ptr(vsum), _ptr(bias), _stream(stream)),
+           "bsa_summarize_permuted")
 
 
 def bsa_permute(p, Q, K, V, perm, Qp, Kp, Vp, stream=None):

@@ -784,6 +784,38 @@ int bsa_permute(const bsa_params* p, const void* Q, const void* K, const void* V
                                               static_cast<cudaStream_t>(stream)));
 }
 
+int bsa_pool_permuted(const bsa_params* p, const void* Q, const int32_t* perm, void* Qp,
+                      float* qpool, float* anchor, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!Q || !perm || !Qp || !qpool || !anchor) return BSA_ERR_INVALID;
+  if (!aligned(Q, 16) || !aligned(Qp, 16) || !aligned(perm, 4) || !aligned(qpool, 16) ||
+      !aligned(anchor, 16))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return cuda_status(
+      bsa::launch_pool(s, Q, qpool, anchor, static_cast<cudaStream_t>(stream), perm, Qp));
+}
+
+int bsa_summarize_permuted(const bsa_params* p, const void* K, const void* V,
+                           const int32_t* perm, void* Kp, void* Vp, const float* anchor,
+                           float* kpool, void* ksum, void* vsum, float* bias, void* stream) {
+  Shape s;
+  int rc = shape_of(p, &s);
+  if (rc) return rc;
+  if (!K || !V || !perm || !Kp || !Vp || !kpool || !ksum || !vsum || !bias) return BSA_ERR_INVALID;
+  if (s.variant == BSA_SUMMARY_ANCHOR && !anchor) return BSA_ERR_INVALID;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(Kp, 16) || !aligned(Vp, 16) ||
+      !aligned(perm, 4) || !aligned(kpool, 16) || !aligned(ksum, 16) || !aligned(vsum, 16) ||
+      !aligned(bias, 4) || (anchor && !aligned(anchor, 16)))
+    return BSA_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return cuda_status(bsa::launch_summarize(s, K, V, anchor, kpool, ksum, vsum, bias,
+                                           static_cast<cudaStream_t>(stream), nullptr, nullptr,
+                                           nullptr, perm, Kp, Vp));
+}
+
 int bsa_unpermute(const bsa_params* p, const void* Op, const float* lsep, const int32_t* perm,
                   void* O, float* lse, void* stream) {
   Shape s;
@@ -820,12 +852,15 @@ int bsa_forward_reblock(const bsa_params* p, const void* Q, const void* K, const
   reblock_forward_carve(s, static_cast<uint8_t*>(workspace), &w);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = reblock_impl(s, Q, K, w.perm, w.rb, st))) return rc;
-  if ((rc = cuda_status(bsa::launch_permute_rows(s, Q, K, V, w.perm, w.Qp, w.Kp, w.Vp, st))))
-    return rc;
   Workspace fw;
   carve(s, w.fw, &fw);
-  if ((rc = pool_impl(s, w.Qp, fw.qpool, fw.anchor, st))) return rc;
-  if ((rc = summarize_impl(s, w.Kp, w.Vp, fw.anchor, fw.kpool, fw.ksum, fw.vsum, fw.bias, st)))
+  // pool and summarize read Q, K, V through the permutation and write the
+  // permuted rows the attention reads (no separate gather pass)
+  if ((rc = cuda_status(bsa::launch_pool(s, Q, fw.qpool, fw.anchor, st, w.perm, w.Qp))))
+    return rc;
+  if ((rc = cuda_status(bsa::launch_summarize(s, K, V, fw.anchor, fw.kpool, fw.ksum, fw.vsum,
+                                              fw.bias, st, nullptr, nullptr, nullptr, w.perm,
+                                              w.Kp, w.Vp))))
     return rc;
   if ((rc = select_impl(s, fw.qpool, fw.kpool, fw.idx, fw.cnt, st))) return rc;
   if ((rc = attend_impl(s, w.Qp, w.Kp, w.Vp, fw.idx, fw.cnt, fw.ksum, fw.vsum, fw.bias, w.Op,

@@ -38,15 +38,19 @@ struct Shape {
   int* dev_status;  // optional
 };
 
+// perm / Qp (optional): pool the permuted layout (row i of a head is Q row
+// perm[i] of that head), writing the permuted rows to Qp.
 cudaError_t launch_pool(const Shape& s, const void* Q, float* qpool, float* anchor,
-                        cudaStream_t st);
+                        cudaStream_t st, const int32_t* perm = nullptr, void* Qp = nullptr);
 // kstat / vstat / lse_blk (optional, all or none): fp32 k~ and v~ (anchor
 // variant) or mean k and mean v (mean variant), [B,H,nb,128], and the block
-// LSE at the anchor (ln n for the mean variant), [B,H,nb].
+// LSE at the anchor (ln n for the mean variant), [B,H,nb].  perm / Kp / Vp
+// (optional): summarize the permuted layout, writing its K and V rows.
 cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const float* anchor,
                              float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st,
                              float* kstat = nullptr, float* vstat = nullptr,
-                             float* lse_blk = nullptr);
+                             float* lse_blk = nullptr, const int32_t* perm = nullptr,
+                             void* Kp = nullptr, void* Vp = nullptr);
 // Selection.  With `maps` (fp32 qpool / kpool as [BH, nb, 128] with 128-byte
 // swizzle, boxes {32, select_tc_rows(s), 1} and {32, 128, 1}) and
 // select_tc_rows(s) > 0 (rows of up to 3072 video blocks) the scores come

@@ -2,6 +2,10 @@
 //
 //  pool_q_kernel       one CTA per (query block, head): reads the block's
 //                      128 x 128 bf16 rows once, writes its fp32 mean (qpool).
+//                      On a permuted (reblocked) layout it reads the rows
+//                      through the permutation and also writes them out in
+//                      the new order (summarize_kernel does the same for K
+//                      and V), so the layout costs no separate gather pass.
 //  anchor_kernel       one CTA per head: q-bar = mean of the video query rows
 //                      ("the mean of the video queries as one anchor per
 //                      head", Spark-H3 page, Spark-Reweight bullet), summed
@@ -35,6 +39,32 @@ __device__ __forceinline__ void load_block_rows(const __nv_bfloat16* base, int n
   }
 }
 
+// The same rows on a permuted layout: row r of the block is row perm[row0 + r]
+// of the head (clamped into the head), and each loaded chunk is also stored
+// at row row0 + r of `out` (the permuted copy the attention reads).
+__device__ __forceinline__ void load_block_rows_perm(const __nv_bfloat16* head,
+                                                     const int32_t* perm_head, int row0, int n,
+                                                     int N, int g, int c, uint4 rows[8],
+                                                     __nv_bfloat16* out_head) {
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = g + 16 * it;
+    if (r < n) {
+      const int src = min(max(__ldg(perm_head + row0 + r), 0), N - 1);
+      rows[it] = ld_stream_v4(head + static_cast<size_t>(src) * kDim + c * 8);
+    } else {
+      rows[it] = zero;
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = g + 16 * it;
+    if (r < n)
+      *reinterpret_cast<uint4*>(out_head + static_cast<size_t>(row0 + r) * kDim + c * 8) = rows[it];
+  }
+}
+
 // Sum of 8-float vectors over the 16 row groups of the CTA.  Each thread
 // passes its partial for dims [8c, 8c+8); thread d < 128 gets dim d's total.
 // `red` is [8 warps][128] floats of shared memory.  Fixed order: xor-16 pair
@@ -58,9 +88,13 @@ __device__ __forceinline__ float cta_sum_over_rows(const float part[8], float* r
   return s;
 }
 
+// kPerm: pool the permuted layout, reading Q through perm and writing the
+// permuted rows to Qp.
+template <bool kPerm>
 __global__ void __launch_bounds__(kThreads) pool_q_kernel(const __nv_bfloat16* __restrict__ Q,
                                                           float* __restrict__ qpool, int N,
-                                                          int nb) {
+                                                          int nb, const int32_t* __restrict__ perm,
+                                                          __nv_bfloat16* __restrict__ Qp) {
   __shared__ float red[8 * kDim];
   const int blk = blockIdx.x;
   const size_t bh = blockIdx.y;
@@ -68,7 +102,11 @@ __global__ void __launch_bounds__(kThreads) pool_q_kernel(const __nv_bfloat16* _
   const int n = min(kBlock, N - row0);
   const int g = threadIdx.x >> 4, c = threadIdx.x & 15;
   uint4 rows[8];
-  load_block_rows(Q + (bh * N + row0) * kDim, n, g, c, rows);
+  if constexpr (kPerm)
+    load_block_rows_perm(Q + bh * N * kDim, perm + bh * N, row0, n, N, g, c, rows,
+                         Qp + bh * N * kDim);
+  else
+    load_block_rows(Q + (bh * N + row0) * kDim, n, g, c, rows);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int it = 0; it < 8; ++it) {
@@ -104,12 +142,15 @@ __global__ void __launch_bounds__(1024) anchor_kernel(const float* __restrict__ 
   }
 }
 
-template <int kVariant>  // 0 = anchor-weighted, 1 = mean-pooled
+// kVariant: 0 = anchor-weighted, 1 = mean-pooled; kPerm: the permuted layout
+template <int kVariant, bool kPerm>
 __global__ void __launch_bounds__(kThreads) summarize_kernel(
     const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
     const float* __restrict__ anchor, float* __restrict__ kpool, __nv_bfloat16* __restrict__ ksum,
     __nv_bfloat16* __restrict__ vsum, float* __restrict__ bias, float* __restrict__ kstat,
-    float* __restrict__ vstat, float* __restrict__ lse_blk, int N, int nb, float scale) {
+    float* __restrict__ vstat, float* __restrict__ lse_blk, int N, int nb, float scale,
+    const int32_t* __restrict__ perm, __nv_bfloat16* __restrict__ Kp,
+    __nv_bfloat16* __restrict__ Vp) {
   __shared__ float red[8 * kDim];
   __shared__ float xs[kBlock];
   __shared__ float stat[2];
@@ -121,8 +162,15 @@ __global__ void __launch_bounds__(kThreads) summarize_kernel(
   const int lane = tid & 31, warp = tid >> 5;
 
   uint4 kr[8], vr[8];
-  load_block_rows(K + (bh * N + row0) * kDim, n, g, c, kr);
-  load_block_rows(V + (bh * N + row0) * kDim, n, g, c, vr);
+  if constexpr (kPerm) {   // K and V through perm, their copies to Kp, Vp
+    load_block_rows_perm(K + bh * N * kDim, perm + bh * N, row0, n, N, g, c, kr,
+                         Kp + bh * N * kDim);
+    load_block_rows_perm(V + bh * N * kDim, perm + bh * N, row0, n, N, g, c, vr,
+                         Vp + bh * N * kDim);
+  } else {
+    load_block_rows(K + (bh * N + row0) * kDim, n, g, c, kr);
+    load_block_rows(V + (bh * N + row0) * kDim, n, g, c, vr);
+  }
 
   float ks[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -242,29 +290,47 @@ __global__ void __launch_bounds__(kThreads) summarize_kernel(
 }  // namespace
 
 cudaError_t launch_pool(const Shape& s, const void* Q, float* qpool, float* anchor,
-                        cudaStream_t st) {
+                        cudaStream_t st, const int32_t* perm, void* Qp) {
   const dim3 grid(s.nb, s.B * s.H);
-  pool_q_kernel<<<grid, kThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(Q), qpool, s.N,
-                                           s.nb);
+  if (perm)
+    pool_q_kernel<true><<<grid, kThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(Q), qpool,
+                                                   s.N, s.nb, perm,
+                                                   static_cast<__nv_bfloat16*>(Qp));
+  else
+    pool_q_kernel<false><<<grid, kThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(Q), qpool,
+                                                    s.N, s.nb, nullptr, nullptr);
   anchor_kernel<<<s.B * s.H, 1024, 0, st>>>(qpool, anchor, s.N, s.nb, s.pb);
   return cudaGetLastError();
 }
 
 cudaError_t launch_summarize(const Shape& s, const void* K, const void* V, const float* anchor,
                              float* kpool, void* ksum, void* vsum, float* bias, cudaStream_t st,
-                             float* kstat, float* vstat, float* lse_blk) {
+                             float* kstat, float* vstat, float* lse_blk, const int32_t* perm,
+                             void* Kp_out, void* Vp_out) {
   const dim3 grid(s.nb, s.B * s.H);
   const float scale = 0.088388347648318440550f;  // 1 / sqrt(128)
   auto Kp = static_cast<const __nv_bfloat16*>(K);
   auto Vp = static_cast<const __nv_bfloat16*>(V);
   auto ks = static_cast<__nv_bfloat16*>(ksum);
   auto vs = static_cast<__nv_bfloat16*>(vsum);
-  if (s.variant == 0)
-    summarize_kernel<0><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias, kstat,
-                                                   vstat, lse_blk, s.N, s.nb, scale);
+  auto ko = static_cast<__nv_bfloat16*>(Kp_out);
+  auto vo = static_cast<__nv_bfloat16*>(Vp_out);
+  if (s.variant == 0 && perm)
+    summarize_kernel<0, true><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias,
+                                                         kstat, vstat, lse_blk, s.N, s.nb, scale,
+                                                         perm, ko, vo);
+  else if (s.variant == 0)
+    summarize_kernel<0, false><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias,
+                                                          kstat, vstat, lse_blk, s.N, s.nb, scale,
+                                                          nullptr, nullptr, nullptr);
+  else if (perm)
+    summarize_kernel<1, true><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias,
+                                                         kstat, vstat, lse_blk, s.N, s.nb, scale,
+                                                         perm, ko, vo);
   else
-    summarize_kernel<1><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias, kstat,
-                                                   vstat, lse_blk, s.N, s.nb, scale);
+    summarize_kernel<1, false><<<grid, kThreads, 0, st>>>(Kp, Vp, anchor, kpool, ks, vs, bias,
+                                                          kstat, vstat, lse_blk, s.N, s.nb, scale,
+                                                          nullptr, nullptr, nullptr);
   return cudaGetLastError();
 }
 

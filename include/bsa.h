@@ -248,6 +248,21 @@ int bsa_reblock(const bsa_params* p, const void* Q, const void* K, int32_t* perm
 int bsa_permute(const bsa_params* p, const void* Q, const void* K, const void* V,
                 const int32_t* perm, void* Qp, void* Kp, void* Vp, void* stream);
 
+/* bsa_permute of Q followed by bsa_pool on Qp, in one pass: Qp[b,h,i] =
+ * Q[b,h,perm[b,h,i]] is written and the pooled means (qpool, anchor) are
+ * those of the reblocked layout, bit for bit what the two calls give.  perm
+ * is bsa_reblock's permutation of [0, N) per (b, h) (an entry outside [0, N)
+ * is clamped into it).  Q, Qp 16-byte aligned; Qp must not overlap Q. */
+int bsa_pool_permuted(const bsa_params* p, const void* Q, const int32_t* perm, void* Qp,
+                      float* qpool, float* anchor, void* stream);
+
+/* bsa_permute of K and V followed by bsa_summarize on Kp, Vp, in one pass:
+ * writes Kp, Vp and the summaries of the reblocked layout, bit for bit what
+ * the two calls give.  Same perm contract as bsa_pool_permuted. */
+int bsa_summarize_permuted(const bsa_params* p, const void* K, const void* V,
+                           const int32_t* perm, void* Kp, void* Vp, const float* anchor,
+                           float* kpool, void* ksum, void* vsum, float* bias, void* stream);
+
 /* O[b,h,perm[b,h,i]] = Op[b,h,i] (and lse from lsep when lse is non-NULL):
  * back to the original token order. */
 int bsa_unpermute(const bsa_params* p, const void* Op, const float* lsep, const int32_t* perm,
@@ -257,8 +272,9 @@ int bsa_unpermute(const bsa_params* p, const void* Op, const float* lsep, const 
  * reblocking scratch and the forward's workspace. */
 size_t bsa_forward_reblock_workspace_bytes(const bsa_params* p);
 
-/* bsa_reblock, bsa_permute, bsa_forward (pool, summarize, select, attend) on
- * the reblocked layout, bsa_unpermute: O (and lse) in the original order. */
+/* bsa_reblock, then bsa_pool_permuted and bsa_summarize_permuted (the
+ * reblocked layout without a separate gather), bsa_select and bsa_attend on
+ * it, bsa_unpermute: O (and lse) in the original order. */
 int bsa_forward_reblock(const bsa_params* p, const void* Q, const void* K, const void* V,
                         void* O, float* lse, void* workspace, size_t workspace_bytes,
                         void* stream);

@@ -123,6 +123,12 @@ def test_option_arguments_rejected_before_launch():
     assert L.bsa_reblock(P, a, a, a, a, 16, None) == bsa.BSA_ERR_INVALID      # scratch too small
     assert L.bsa_reblock(P, odd, a, a, a, 1 << 40, None) == bsa.BSA_ERR_ALIGN
     assert L.bsa_permute(P, a, a, a, None, a, a, a, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_pool_permuted(P, a, None, a, a, a, None) == bsa.BSA_ERR_INVALID
+    assert L.bsa_pool_permuted(P, a, a, odd, a, a, None) == bsa.BSA_ERR_ALIGN       # Qp
+    assert L.bsa_summarize_permuted(P, a, a, None, a, a, a, a, a, a, a, None) == \
+        bsa.BSA_ERR_INVALID
+    assert L.bsa_summarize_permuted(P, a, a, a, a, odd, a, a, a, a, a, None) == \
+        bsa.BSA_ERR_ALIGN                                                             # Vp
     assert L.bsa_unpermute(P, a, None, a, a, a, None) == bsa.BSA_ERR_INVALID   # lse without lsep
     assert L.bsa_forward_reblock(P, a, a, a, a, None, a, 16, None) == bsa.BSA_ERR_INVALID
     # FP8

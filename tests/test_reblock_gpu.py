@@ -156,3 +156,32 @@ def test_reblock_full_size_sampled_head():
     assert torch.equal(O[:, h:h + 1], Ob)
     del Q, K, V, O
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("N,prefix,variant", [(1500, 256, "anchor"), (4100, 0, "mean"),
+                                              (17_000, 0, "anchor")])
+def test_permuted_stages_equal_permute_then_stages(N, prefix, variant):
+    # bsa_pool_permuted / bsa_summarize_permuted read through perm and write
+    # the permuted rows themselves: the same bits as bsa_permute followed by
+    # bsa_pool / bsa_summarize on the permuted copies
+    B, H = 1, 2
+    Q, K, V = make_qkv(B, H, N, 128, "block_offset", 4, device="cuda")
+    p = bsa.params(B, H, N, 8, prefix, variant)
+    perm = torch.empty(B, H, N, dtype=torch.int32, device="cuda")
+    ws = torch.empty(max(256, bsa.bsa_reblock_workspace_bytes(p)), dtype=torch.uint8,
+                     device="cuda")
+    bsa.bsa_reblock(p, Q, K, perm, ws)
+    Qp, Kp, Vp = (torch.empty_like(X) for X in (Q, K, V))
+    bsa.bsa_permute(p, Q, K, V, perm, Qp, Kp, Vp)
+    a = bsa.stage_buffers(B, H, N, 8, prefix, variant)
+    bsa.bsa_pool(p, Qp, a["qpool"], a["anchor"])
+    bsa.bsa_summarize(p, Kp, Vp, a["anchor"], a["kpool"], a["ksum"], a["vsum"], a["bias"])
+    b = bsa.stage_buffers(B, H, N, 8, prefix, variant)
+    Qq, Kq, Vq = (torch.full_like(X, float("nan")) for X in (Q, K, V))
+    bsa.bsa_pool_permuted(p, Q, perm, Qq, b["qpool"], b["anchor"])
+    bsa.bsa_summarize_permuted(p, K, V, perm, Kq, Vq, b["anchor"], b["kpool"], b["ksum"],
+                               b["vsum"], b["bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(Qq, Qp) and torch.equal(Kq, Kp) and torch.equal(Vq, Vp)
+    for k in ("qpool", "anchor", "kpool", "ksum", "vsum", "bias"):
+        assert torch.equal(a[k], b[k]), k
