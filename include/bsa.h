@@ -145,7 +145,7 @@ int bsa_forward(const bsa_params* p, const void* Q, const void* K, const void* V
 /* bsa_forward from HOST buffers.  hQ, hK, hV (bf16 [B,H,N,D]) are copied to
  * the caller's device buffers dQ, dK, dV, the forward runs, and dO is copied
  * back to hO (and dlse to hlse when both are non-NULL).  The work is
- * pipelined over up to 8 chunks of (b, h) slices: the host->device copies
+ * pipelined over up to 16 chunks of (b, h) slices: the host->device copies
  * (one cudaMemcpyAsync per tensor and chunk) run on a helper stream, the
  * forward of each chunk on `stream`, the copies back on a second helper
  * stream, ordered by events, so copies overlap compute and each other.
