@@ -95,9 +95,9 @@ def parse_args():
 def reblock_launches(N: int, prefix: int) -> int:
     """Kernels bsa_reblock launches (its tree shape depends on N - prefix only):
     init + key moment (Gram, reduction) + factor + whiten, then per level a
-    Gram and a split, a projection on levels whose largest group exceeds 384
-    rows (smaller groups are projected in their Gram CTA), and a partial-sum
-    pass on levels whose largest group spans more than one 2048-row chunk."""
+    Gram and a split, plus a partial-sum pass and a projection on levels whose
+    largest group spans more than one 2048-row chunk (single-chunk groups are
+    projected in their Gram CTA)."""
     nv = N - prefix
     levels = 0
     while (128 << levels) < nv:
@@ -106,7 +106,7 @@ def reblock_launches(N: int, prefix: int) -> int:
         return 1
     n, largest = 5, nv
     for _ in range(levels):
-        n += 2 + (1 if largest > 384 else 0) + (1 if largest > 2048 else 0)
+        n += 2 + (2 if largest > 2048 else 0)
         largest -= ((largest + 127) // 128 // 2) * 128
     return n
 

@@ -35,9 +35,10 @@
 //                         CTA, larger groups leave partials for group_kernel.
 //   group_kernel          fixed-order sum of a large group's partials, power
 //                         iteration.
-//   project_kernel        p = u . v per position -> order-preserving key
-//                         (groups of at most 3 tiles: in their Gram CTA,
-//                         whose ring still holds all their rows).
+//   project_kernel        p = u . v per position -> order-preserving key, for
+//                         groups of several chunks (a single-chunk group is
+//                         projected by its Gram CTA: from the ring, or for more
+//                         than 3 tiles from a second pass over its rows).
 //   split_kernel          radix select of the floor(b/2)*128-th key (four
 //                         8-bit passes over the group's keys, ties broken by
 //                         position), then a stable partition of perm
@@ -139,8 +140,10 @@ struct GramArgs {
 
 constexpr int kStages = 3;   // Gram tiles in flight (cp.async ring)
 constexpr uint32_t kGramCols = 256;   // TMEM: Gram in columns 0-127, column sums 128-143
-// Groups of at most this many rows stay whole in the Gram CTA's ring, which
-// then also forms their projections (project_kernel skips them).
+// Groups of at most this many rows stay whole in the Gram CTA's ring; the
+// CTA forms their projections from it.  Larger single-chunk groups stream
+// their rows through the ring once more for the projections (from L2), and
+// project_kernel takes only the groups of several chunks.
 constexpr int kGramProjRows = kStages * kBlock;
 
 struct GramSmem {
@@ -294,30 +297,44 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
       __syncthreads();
       power_iterate(gr, n, ctl->c, ctl->v, ctl->red,
                     a.vdir + (bh * a.slots + slot) * kDim);
-      if (g.count <= kGramProjRows) {
-        // p = u . v of every row (tile it sits in buffer it: ntile <= kStages),
-        // summed in project_kernel's order: eight products per 16-byte chunk,
-        // then the chunks pairwise as its lane butterfly does
-        for (int it = 0; it < ntile; ++it) {
-          const int pos = p0 + it * kBlock + tid;
-          if (pos >= p1) break;
-          const uint8_t* buf = sm + it * kTile;
-          float part[16];
+      // p = u . v of every row of the group, summed in project_kernel's
+      // order: eight products per 16-byte chunk, then the chunks pairwise as
+      // its lane butterfly does.  Thread tid takes row tid of each tile.
+      auto project_tile = [&](const uint8_t* buf, int it) {
+        const int pos = p0 + it * kBlock + tid;
+        if (pos >= p1) return;
+        float part[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const uint4 w = *reinterpret_cast<const uint4*>(buf + swz(tid, c));
-            const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&w);
-            float sc = 0.f;
+        for (int c = 0; c < 16; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(buf + swz(tid, c));
+          const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&w);
+          float sc = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sc = fmaf(__bfloat162float(h[e]), ctl->v[8 * c + e], sc);
-            part[c] = sc;
-          }
-#pragma unroll
-          for (int o = 8; o > 0; o >>= 1)
-#pragma unroll
-            for (int c = 0; c < o; ++c) part[c] = part[c] + part[c + o];
-          a.keys[bh * a.nv + pos] = orderable_key(part[0]);
+          for (int e = 0; e < 8; ++e) sc = fmaf(__bfloat162float(h[e]), ctl->v[8 * c + e], sc);
+          part[c] = sc;
         }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+          for (int c = 0; c < o; ++c) part[c] = part[c] + part[c + o];
+        a.keys[bh * a.nv + pos] = orderable_key(part[0]);
+      };
+      if (g.count <= kGramProjRows) {
+        // every tile is still in the ring (tile it in buffer it)
+        for (int it = 0; it < ntile; ++it) project_tile(sm + it * kTile, it);
+      } else {
+        // stream the group's rows through the ring once more (they were just
+        // read, so they come from L2)
+        issue_tile(0);
+        issue_tile(1);
+        for (int it = 0; it < ntile; ++it) {
+          __syncthreads();   // buffer (it + 2) % kStages (tile it - 1) is done with
+          issue_tile(it + 2);
+          cp_async_wait<2>();
+          __syncthreads();
+          project_tile(sm + (it % kStages) * kTile, it);
+        }
+        cp_async_wait<0>();
       }
     } else {
       float4* dst = reinterpret_cast<float4*>(a.part + (pidx * 128 + tid) * 128);
@@ -638,7 +655,7 @@ __global__ void __launch_bounds__(256) project_kernel(const __nv_bfloat16* __res
   const int slot = blockIdx.x / max_pchunks, chunk = blockIdx.x - slot * max_pchunks;
   const size_t bh = blockIdx.y;
   const Range g = group_of(nv, level, slot);
-  if (g.count <= kGramProjRows) return;   // leaves; small groups are done in the Gram CTA
+  if (g.count <= kChunkTok) return;   // leaves; single-chunk groups are done in their Gram CTA
   const int p0 = g.start + chunk * kProjTok, p1 = min(p0 + kProjTok, g.start + g.count);
   if (p0 >= p1) return;
   if (tid < 128) v[tid] = vdir[(bh * slots + slot) * kDim + tid];
@@ -897,8 +914,8 @@ ReblockPlan reblock_plan(const Shape& s) {
     const int chunks = (largest + kChunkTok - 1) / kChunkTok;
     p.max_chunks[l] = chunks;
     // the rightmost group is the largest: none left for project_kernel when
-    // it fits in a Gram CTA's ring
-    p.max_pchunks[l] = largest > kGramProjRows ? (largest + kProjTok - 1) / kProjTok : 0;
+    // it fits in one Gram chunk
+    p.max_pchunks[l] = largest > kChunkTok ? (largest + kProjTok - 1) / kProjTok : 0;
     p.largest[l] = largest;
     const long long parts = (chunks > 1) ? (static_cast<long long>(1) << l) * chunks : 1;
     if (parts > p.max_partials) p.max_partials = static_cast<int>(parts);
