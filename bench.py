@@ -95,9 +95,10 @@ def parse_args():
 def reblock_launches(N: int, prefix: int) -> int:
     """Kernels bsa_reblock launches (its tree shape depends on N - prefix only):
     init + key moment (Gram, reduction) + factor + whiten, then per level a
-    Gram and a split, plus a partial-sum pass and a projection on levels whose
-    largest group spans more than one 2048-row chunk (single-chunk groups are
-    projected in their Gram CTA)."""
+    Gram and a split, plus a power-iteration pass and a projection on levels
+    whose largest group spans more than one 2048-row chunk (single-chunk
+    groups finish in their Gram CTA) and a partial-sum reduction where it
+    spans four or more."""
     nv = N - prefix
     levels = 0
     while (128 << levels) < nv:
@@ -106,7 +107,8 @@ def reblock_launches(N: int, prefix: int) -> int:
         return 1
     n, largest = 5, nv
     for _ in range(levels):
-        n += 2 + (2 if largest > 2048 else 0)
+        chunks = (largest + 2047) // 2048
+        n += 2 + (2 if chunks > 1 else 0) + (1 if chunks >= 4 else 0)
         largest -= ((largest + 127) // 128 // 2) * 128
     return n
 

@@ -33,8 +33,9 @@
 //                         rows (gathered through perm); a group that fits in
 //                         one chunk finishes its power iteration in the same
 //                         CTA, larger groups leave partials for group_kernel.
-//   group_kernel          fixed-order sum of a large group's partials, power
-//                         iteration.
+//   group_reduce_kernel   fixed-order sum of a large group's partials, one
+//                         CTA per row of its Gram;
+//   group_kernel          then its power iteration.
 //   project_kernel        p = u . v per position -> order-preserving key, for
 //                         groups of several chunks (a single-chunk group is
 //                         projected by its Gram CTA: from the ring, or for more
@@ -135,6 +136,7 @@ struct GramArgs {
   float* psum;              // [BH, slots * max_chunks, 128]  (group mode)
   float* vdir;              // [BH, slots, 128]                (group mode)
   uint32_t* keys;           // [BH, nv] projection keys of small groups (group mode)
+  int reduced;              // group_reduce_kernel has summed the partials of this level
   int* dev_status;
 };
 
@@ -353,8 +355,34 @@ __global__ void __launch_bounds__(128) gram_kernel(const GramArgs a) {
   }
 }
 
-// Power iteration of a group larger than one chunk: fixed-order sum of its
-// chunk partials.
+// Fixed-order sum of a large group's chunk partials, one CTA per row of its
+// Gram (blockIdx.x < 128; the column sums for blockIdx.x == 128), left in the
+// group's first partial slot: thread j adds element j of the row chunk by
+// chunk, so the sums are those a single thread per row would form.
+__global__ void __launch_bounds__(128) group_reduce_kernel(const GramArgs a) {
+  const int r = blockIdx.x, slot = blockIdx.y, j = threadIdx.x;
+  const size_t bh = blockIdx.z;
+  const Range g = group_of(a.nv, a.level, slot);
+  if (g.count <= kChunkTok) return;   // leaves and single-chunk groups are done
+  const int nch = (g.count + kChunkTok - 1) / kChunkTok;
+  const size_t p0 = static_cast<size_t>(bh) * a.slots * a.max_chunks +
+                    static_cast<size_t>(slot) * a.max_chunks;
+  float acc = 0.f;
+  if (r < 128) {
+#pragma unroll 4
+    for (int ch = 0; ch < nch; ++ch) acc += __ldg(a.part + ((p0 + ch) * 128 + r) * 128 + j);
+    a.part[(p0 * 128 + r) * 128 + j] = acc;
+  } else {
+#pragma unroll 4
+    for (int ch = 0; ch < nch; ++ch) acc += __ldg(a.psum + (p0 + ch) * 128 + j);
+    a.psum[p0 * 128 + j] = acc;
+  }
+}
+
+// Power iteration of a group larger than one chunk: on the sums
+// group_reduce_kernel left in its first partial slot (a.reduced), or summing
+// the chunk partials itself in the same order (groups of a few chunks, where
+// a CTA per row would be mostly launch cost).
 __global__ void __launch_bounds__(128) group_kernel(const GramArgs a) {
   __shared__ alignas(16) float c[128];
   __shared__ alignas(16) float v[128];
@@ -363,13 +391,13 @@ __global__ void __launch_bounds__(128) group_kernel(const GramArgs a) {
   const size_t bh = blockIdx.y;
   const Range g = group_of(a.nv, a.level, slot);
   if (g.count <= kChunkTok) return;   // leaves and single-chunk groups are done
-  const int nch = (g.count + kChunkTok - 1) / kChunkTok;
   float gr[128];
 #pragma unroll
   for (int j = 0; j < 128; ++j) gr[j] = 0.f;
   float s = 0.f;
   const size_t p0 = static_cast<size_t>(bh) * a.slots * a.max_chunks +
                     static_cast<size_t>(slot) * a.max_chunks;
+  const int nch = a.reduced ? 1 : (g.count + kChunkTok - 1) / kChunkTok;
   // chunk by chunk in a fixed order; each chunk's row arrives as 32
   // independent 16-byte loads issued together
   for (int ch = 0; ch < nch; ++ch) {
@@ -1001,7 +1029,13 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
     ga.slots = slots;
     ga.max_chunks = plan.max_chunks[l];
     gram_kernel<true><<<dim3(slots * plan.max_chunks[l], BH), 128, gram_smem, st>>>(ga);
-    if (plan.max_chunks[l] > 1) group_kernel<<<dim3(slots, BH), 128, 0, st>>>(ga);
+    if (plan.max_chunks[l] > 1) {
+      // a CTA per Gram row for groups of 4 or more chunks (768p-5s level 0,
+      // 18 chunks: 67 -> 28 us); a CTA per group below that
+      ga.reduced = plan.max_chunks[l] >= 4 ? 1 : 0;
+      if (ga.reduced) group_reduce_kernel<<<dim3(129, slots, BH), 128, 0, st>>>(ga);
+      group_kernel<<<dim3(slots, BH), 128, 0, st>>>(ga);
+    }
     if (plan.max_pchunks[l] > 0)
       project_kernel<<<dim3(slots * plan.max_pchunks[l], BH), 256, 0, st>>>(
           w.u, pa, w.vdir, s.N, s.prefix, nv, l, slots, plan.max_pchunks[l], w.keys);
