@@ -505,16 +505,17 @@ int attend_extra_impl(const Shape& s, int n_extra, const void* Q, const void* K,
                                               side_bias, side_cnt, scap, O, lse, st));
 }
 
-// A forward from HOST buffers, pipelined over chunks of (b, h) slices; `fwd`
-// runs the forward of one chunk (a sub-call with B = 1) on the caller's
-// stream with the caller's workspace, which a sub-call needs no more of than
-// the whole call.  Validates the pointers of the device side before the first
-// copy, so an argument error enqueues nothing.
+// A forward from HOST buffers, pipelined over up to `max_chunks` chunks of
+// (b, h) slices; `fwd` runs the forward of one chunk (a sub-call with B = 1)
+// on the caller's stream with the caller's workspace, which a sub-call needs
+// no more of than the whole call.  Validates the pointers of the device side
+// before the first copy, so an argument error enqueues nothing.
+constexpr int kMaxChunks = 16;
 template <class Fwd>
 int forward_host_pipelined(const bsa_params* p, const void* hQ, const void* hK, const void* hV,
                            void* hO, float* hlse, void* dQ, void* dK, void* dV, void* dO,
                            float* dlse, void* workspace, size_t workspace_bytes, void* stream,
-                           Fwd fwd) {
+                           Fwd fwd, int max_chunks = kMaxChunks) {
   Shape s;
   int rc = shape_of(p, &s);
   if (rc) return rc;
@@ -534,12 +535,12 @@ int forward_host_pipelined(const bsa_params* p, const void* hQ, const void* hK, 
   // waits for the last copy, so synchronising it covers everything.
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = s.B * s.H;
-  // up to 16 chunks: the last chunk's forward and copy back are what the
-  // pipeline cannot hide (measured at 56 heads: 33.5 / 119.6 ms with 8 chunks,
-  // 32.9 / 115.8 with 14 of 4 heads, 33.2 / 114.3 with 28 of 2, for 768p-5s /
-  // 2K-5s)
-  constexpr int kMaxChunks = 16;
-  const int nchunk = BH < kMaxChunks ? BH : kMaxChunks;
+  // up to 16 chunks by default: the last chunk's forward and copy back are
+  // what the pipeline cannot hide (measured at 56 heads: 33.5 / 119.6 ms with
+  // 8 chunks, 32.9 / 115.8 with 14 of 4 heads, 33.2 / 114.3 with 28 of 2, for
+  // 768p-5s / 2K-5s)
+  const int cap = max_chunks < 1 ? 1 : (max_chunks > kMaxChunks ? kMaxChunks : max_chunks);
+  const int nchunk = BH < cap ? BH : cap;
   const int per = (BH + nchunk - 1) / nchunk;
   const size_t slice = static_cast<size_t>(s.N) * 128 * 2;     // bytes of one (b, h) slice
   const size_t lslice = static_cast<size_t>(s.N) * 4;
@@ -1182,7 +1183,11 @@ int bsa_forward_extra_host(const bsa_params* p, int32_t n_extra, const void* hQ,
       [n_extra](const bsa_params* sub, void* q, void* k, void* v, void* o, float* l, void* ws,
                 size_t wsb, void* st) {
         return bsa_forward_extra(sub, n_extra, q, k, v, o, l, ws, wsb, st);
-      });
+      },
+      // 8 chunks: the token selection has a CTA per 128 query blocks, so a
+      // chunk of few heads leaves most SMs idle (measured at 768p-5s: 35.3 ms
+      // per call with 8 chunks, 44.2 with 14)
+      8);
 }
 
 int bsa_forward_reblock_host(const bsa_params* p, const void* hQ, const void* hK,

@@ -166,7 +166,9 @@ int bsa_forward_host(const bsa_params* p, const void* hQ, const void* hK,
  * workspace bsa_forward_extra_workspace_bytes) and adaptive reblocking
  * (bsa_forward_reblock, workspace bsa_forward_reblock_workspace_bytes), each
  * chunk's forward being the option's own forward on a sub-call of its
- * slices.  Arguments, streams and error behaviour as bsa_forward_host. */
+ * slices (up to 8 chunks for extra tokens, whose token selection needs many
+ * heads per launch to fill the GPU).  Arguments, streams and error behaviour
+ * as bsa_forward_host. */
 int bsa_forward_fp8_host(const bsa_params* p, const void* hQ, const void* hK, const void* hV,
                          void* hO, float* hlse, void* dQ, void* dK, void* dV, void* dO,
                          float* dlse, void* workspace, size_t workspace_bytes, void* stream);
