@@ -341,6 +341,9 @@ int reblock_impl(const Shape& s, const void* Q, const void* K, int32_t* perm, ui
   if (!make_map(&maps.q, Q, s.N, bh) || !make_map(&maps.r_hi, w.r_hi, 128, bh) ||
       !make_map(&maps.r_lo, w.r_lo, 128, bh))
     return BSA_ERR_UNSUPPORTED;
+  // the whitened rows (only when there are video tokens to whiten)
+  if (plan.nv > 0 && !make_map(&maps.u, w.u, static_cast<uint64_t>(plan.nv), bh))
+    return BSA_ERR_UNSUPPORTED;
   return cuda_status(bsa::launch_reblock(s, plan, Q, K, maps, w, perm, st));
 }
 

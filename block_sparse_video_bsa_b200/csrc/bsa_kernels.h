@@ -143,6 +143,7 @@ struct ReblockBuffers {
 };
 struct ReblockMaps {
   CUtensorMap q, r_hi, r_lo;   // bf16, box {64, 128, 1}, 128B swizzle
+  CUtensorMap u;               // the whitened rows [BH, nv, 128], same box (TMA stores)
 };
 cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* Q, const void* K,
                            const ReblockMaps& maps, const ReblockBuffers& w, int32_t* perm_out,

@@ -506,10 +506,26 @@ __global__ void __launch_bounds__(128) factor_kernel(const float* __restrict__ M
   }
 }
 
+// AND of `v` over the 128 threads of warps 0-3 (named barrier 1): every one of
+// them gets the same answer, so they leave a loop together.
+__device__ __forceinline__ bool epi_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, 1, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u)
+      : "memory");
+  return r != 0;
+}
+
 constexpr int kWhThreads = 192;   // warps 0-3 epilogue (TMEM lane quarters), 4 TMA, 5 MMA
 constexpr int kWhStages = 3;      // Q tiles in flight
 constexpr uint32_t kWhOffQ = 2 * kTile;                       // after R hi, R lo
-constexpr uint32_t kWhOffCtl = kWhOffQ + kWhStages * kTile;
+constexpr uint32_t kWhOffOut = kWhOffQ + kWhStages * kTile;   // two u tiles for TMA stores
+constexpr uint32_t kWhOffCtl = kWhOffOut + 2 * kTile;
 
 struct WhitenSmem {
   uint64_t rfull, rempty;                   // R (hi + lo) of the current head
@@ -527,8 +543,8 @@ struct WhitenSmem {
 // the MMAs of the next (two accumulators).
 __global__ void __launch_bounds__(kWhThreads, 1)
     whiten_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_hi,
-                  const __grid_constant__ CUtensorMap tm_lo, int prefix, int nv, int ntile,
-                  int total, int per, __nv_bfloat16* __restrict__ u, int* dev_status) {
+                  const __grid_constant__ CUtensorMap tm_lo, const __grid_constant__ CUtensorMap tm_u,
+                  int prefix, int nv, int ntile, int total, int per, int* dev_status) {
   extern __shared__ __align__(1024) uint8_t sm[];
   WhitenSmem* ctl = reinterpret_cast<WhitenSmem*>(sm + kWhOffCtl);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -633,11 +649,14 @@ __global__ void __launch_bounds__(kWhThreads, 1)
       mbar_wait(&ctl->done, 0, wc);
     }
   } else if (run) {
-    // epilogue: thread tid = TMEM lane = token row of the tile
+    // epilogue: thread tid = TMEM lane = token row of the tile; the tile of
+    // u goes to one of two shared buffers in the swizzled layout and leaves
+    // by TMA store (rows past nv are not written)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     for (int it = 0; it < nw; ++it) {
       const int w = w0 + it, bh = w / ntile, tile = w - bh * ntile, b = it & 1;
-      if (!mbar_wait(&ctl->afull[b], (it >> 1) & 1, wc)) break;
+      // all 128 epilogue threads go on or stop together (named barriers below)
+      if (!epi_all(mbar_wait(&ctl->afull[b], (it >> 1) & 1, wc))) break;
       tc_fence_after();
       float y[128];
       BSA_TMEM_LD_32F(tmem + lane_base + b * 128, y);
@@ -647,21 +666,30 @@ __global__ void __launch_bounds__(kWhThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&ctl->aempty[b]);
-      const int t = tile * kBlock + tid;
-      if (t < nv) {
-        float ss = 0.f;
+      float ss = 0.f;
 #pragma unroll
-        for (int j = 0; j < 128; ++j) ss = fmaf(y[j], y[j], ss);
-        const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(u + (static_cast<size_t>(bh) * nv + t) * kDim);
+      for (int j = 0; j < 128; ++j) ss = fmaf(y[j], y[j], ss);
+      const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+      // buffer b was last stored from two tiles ago: that store has read it
+      if (tid == 0) bulk_wait_group_read<1>();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      uint8_t* out = sm + kWhOffOut + b * kTile;
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-          dst[q] = make_uint4(pack_bf16x2(y[8 * q] * inv, y[8 * q + 1] * inv),
-                              pack_bf16x2(y[8 * q + 2] * inv, y[8 * q + 3] * inv),
-                              pack_bf16x2(y[8 * q + 4] * inv, y[8 * q + 5] * inv),
-                              pack_bf16x2(y[8 * q + 6] * inv, y[8 * q + 7] * inv));
+      for (int q = 0; q < 16; ++q)
+        *reinterpret_cast<uint4*>(out + swz(tid, q)) =
+            make_uint4(pack_bf16x2(y[8 * q] * inv, y[8 * q + 1] * inv),
+                       pack_bf16x2(y[8 * q + 2] * inv, y[8 * q + 3] * inv),
+                       pack_bf16x2(y[8 * q + 4] * inv, y[8 * q + 5] * inv),
+                       pack_bf16x2(y[8 * q + 6] * inv, y[8 * q + 7] * inv));
+      fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (tid == 0) {
+        tma_store_3d(out, &tm_u, 0, tile * kBlock, bh);
+        tma_store_3d(out + kHalf, &tm_u, 64, tile * kBlock, bh);
+        bulk_commit_group();
       }
     }
+    if (tid == 0) bulk_wait_group_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -1014,7 +1042,7 @@ cudaError_t launch_reblock(const Shape& s, const ReblockPlan& plan, const void* 
     const int ctas = total < sms ? total : sms;
     const int per = (total + ctas - 1) / ctas;
     whiten_kernel<<<(total + per - 1) / per, kWhThreads, whiten_smem, st>>>(
-        maps.q, maps.r_hi, maps.r_lo, s.prefix, nv, ntile, total, per, w.u, s.dev_status);
+        maps.q, maps.r_hi, maps.r_lo, maps.u, s.prefix, nv, ntile, total, per, s.dev_status);
   }
   (void)Q;
   // 4. levels
