@@ -16,17 +16,20 @@
 //                        split into bf16 hi + lo (qhat ~= hi + lo to ~16 bits;
 //                        K is exact bf16), B = one 128-token key block from
 //                        a 4-stage TMA ring, D = 128 x 128 fp32 in TMEM
-//                        (four buffers).  One thread per query block keeps
-//                        a running threshold and appends the candidates above
-//                        it to its own buffer in global memory as 64-bit keys
-//                        (order-preserving score bits << 32 | ~token, so a
-//                        larger key is a higher score, then a lower index);
+//                        (four buffers).  Two threads per query block, one
+//                        per half of each key block's 128 tokens, each keep a
+//                        running threshold and append the candidates above
+//                        it to their own buffer in global memory as 64-bit
+//                        keys (order-preserving score bits << 32 | ~token, so
+//                        a larger key is a higher score, then a lower index);
 //                        when a buffer fills, the warp compacts it to the
 //                        n_extra largest keys (bitwise binary search with
 //                        warp-wide counts) and raises the threshold to the
 //                        smallest kept key.
 //  extra_finish_kernel   one warp per query block: the n_extra largest keys
-//                        of its buffer, written as tokens in ascending order.
+//                        of its two buffers (each holds the n_extra largest of
+//                        its half, so their union holds the row's), written
+//                        as tokens in ascending order.
 //  extra_summary_kernel  one CTA per video query block: the extra tokens form
 //                        runs by block (the list is ascending); for each
 //                        block that keeps some tokens, its summary over the
@@ -45,9 +48,12 @@ namespace bsa {
 
 namespace {
 
-constexpr int kSelThreads = 192;   // warps 0-3 select, 4 producer, 5 MMA
-constexpr int kSelProducerWarp = 4;
-constexpr int kSelMmaWarp = 5;
+// warps 0-7 select (warp w: TMEM lanes 32 (w % 4) .., token half w / 4),
+// warp 8 producer, warp 9 MMA
+constexpr int kSelWarps = 8;
+constexpr int kSelThreads = 32 * kSelWarps + 64;
+constexpr int kSelProducerWarp = kSelWarps;
+constexpr int kSelMmaWarp = kSelWarps + 1;
 constexpr int kSelRing = 4;
 constexpr uint32_t kTileB = 32768;   // 128 x 128 bf16
 constexpr uint32_t kHalfB = 16384;   // 128 rows x 64 bf16 (one 128-byte swizzle atom wide)
@@ -65,9 +71,12 @@ struct SelCtl {
   uint32_t tmem_base;
   int abort_flag;
   int skip;
+  // each (token half, row) thread's threshold key, read by the row's other
+  // thread: the n_extra-th largest key of either half bounds the row's from below
+  unsigned long long rthr[2][kBlock];
   // per selection warp: the 32 scores of a column group of every lane, [column][lane],
   // read back by the lanes' appends; the compaction's 64-key scratch in between
-  alignas(16) float xs[4][32][32];
+  alignas(16) float xs[kSelWarps][32][32];
 };
 static_assert(kOffSelCtl + sizeof(SelCtl) <= 227 * 1024, "shared memory budget");
 
@@ -75,8 +84,8 @@ struct SelArgs {
   const float* qpool;          // [BH, nb, 128]
   const int32_t* idx;          // [BH, nb, kcap]
   const int32_t* cnt;          // [BH, nb]
-  unsigned long long* cand;    // [BH * nbv, kCap] candidate buffers
-  int32_t* bcnt;               // [BH * nbv] keys left in each buffer
+  unsigned long long* cand;    // [BH * nbv, 2, kCap] candidate buffers (two token halves)
+  int32_t* bcnt;               // [BH * nbv, 2] keys left in each buffer
   int rows_v;                  // BH * nbv
   int32_t* extra;              // [BH, nb, n_extra]
   int32_t* ecnt;               // [BH, nb]
@@ -294,9 +303,10 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }
     for (int b = 0; b < kDBuf; ++b) {
       mbar_init(&ctl->d_full[b], 1);
-      mbar_init(&ctl->d_empty[b], kBlock);
+      mbar_init(&ctl->d_empty[b], 32 * kSelWarps);
     }
     mbar_init(&ctl->fin, 1);
+    for (int e = 0; e < 2 * kBlock; ++e) ctl->rthr[e >> 7][e & (kBlock - 1)] = 0ull;
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
@@ -368,16 +378,17 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   } else {
     // ------------------------------------------------------------ selection
     constexpr int kSlots = kCap / 32;
-    const int r = tid;                        // query block i0 + r, TMEM lane r
+    const int half = warp >> 2;               // tokens 64 half .. 64 half + 63 of each key block
+    const int r = (warp & 3) * 32 + lane;     // query block i0 + r, TMEM lane r
     const bool live = r < rows;
     const int i = i0 + r;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int32_t* lrow = a.idx + (static_cast<size_t>(bh) * a.nb + (live ? i : i0)) * a.kcap;
     const int lcnt = live ? max(1, min(__ldg(a.cnt + static_cast<size_t>(bh) * a.nb + i), a.kcap)) : 0;
     int cur = 0;
     while (cur < lcnt && __ldg(lrow + cur) < a.pb) ++cur;     // the prefix blocks come first
-    unsigned long long* buf =
-        a.cand + (static_cast<size_t>(bh) * a.nbv + (live ? i - a.pb : 0)) * kCap;
+    const size_t brow = (static_cast<size_t>(bh) * a.nbv + (live ? i - a.pb : 0)) * 2 + half;
+    unsigned long long* buf = a.cand + brow * kCap;
     int bcnt = 0;
     unsigned long long thr = 0ull;
     float thf = -INFINITY;
@@ -388,15 +399,21 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       const int j = a.pb + it, b = it % kDBuf;
       if (!sel_wait(&ctl->d_full[b], (it / kDBuf) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      float x[128];
-      const uint32_t dcol = tmem + lane_base + b * 128;
+      float x[64];
+      const uint32_t dcol = tmem + lane_base + b * 128 + 64 * half;
       BSA_TMEM_LD_32F(dcol, x);
       BSA_TMEM_LD_32F(dcol + 32, x + 32);
-      BSA_TMEM_LD_32F(dcol + 64, x + 64);
-      BSA_TMEM_LD_32F(dcol + 96, x + 96);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&ctl->d_empty[b]);
+      if (live) {   // the other half's threshold, when higher (a stale one is merely looser)
+        const unsigned long long o =
+            *reinterpret_cast<volatile unsigned long long*>(&ctl->rthr[half ^ 1][r]);
+        if (o > thr) {
+          thr = o;
+          thf = key_score(o);
+        }
+      }
       bool listed_j = false;
       if (live && cur < lcnt && __ldg(lrow + cur) == j) {
         listed_j = true;
@@ -405,12 +422,13 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       const bool scan = live && !listed_j;
       const int nvalid = (j == a.nb - 1) ? last_n : kBlock;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
+        const int c0 = 64 * half + 32 * q;    // first token of the group within the block
         uint32_t m = 0;
         if (scan) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) m |= (x[32 * q + c] >= thf) ? (1u << c) : 0u;
-          const int lim = nvalid - 32 * q;
+          const int lim = nvalid - c0;
           if (lim < 32) m &= lim > 0 ? ((1u << lim) - 1u) : 0u;
         }
         // every lane walks its own set bits: the lanes append together, each
@@ -425,7 +443,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
           const int c = __ffs(m) - 1;
           m &= m - 1;
           const float xv = xsw[c][lane];
-          const uint32_t u = static_cast<uint32_t>(j * kBlock + 32 * q + c);
+          const uint32_t u = static_cast<uint32_t>(j * kBlock + c0 + c);
           const unsigned long long key =
               (static_cast<unsigned long long>(orderable_key(xv)) << 32) |
               static_cast<uint32_t>(~u);
@@ -444,14 +462,17 @@ __global__ void __launch_bounds__(kSelThreads, 1)
             rb, count, a.n_extra, reinterpret_cast<unsigned long long*>(&xsw[0][0]));
         if (lane == L) {
           bcnt = a.n_extra;
-          thr = t;
-          thf = key_score(t);
+          if (t > thr) {
+            thr = t;
+            thf = key_score(t);
+          }
+          *reinterpret_cast<volatile unsigned long long*>(&ctl->rthr[half][r]) = thr;
         }
       }
     }
     // the buffer's fill count goes to the finishing kernel, which keeps the
     // n_extra largest keys and writes them ascending by token
-    if (live) a.bcnt[static_cast<size_t>(bh) * a.nbv + (i - a.pb)] = ok ? bcnt : 0;
+    if (live) a.bcnt[brow] = ok ? bcnt : 0;
   }
 
   tc_fence_before();
@@ -463,8 +484,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   }
 }
 
-// One warp per video query block: the n_extra largest keys of its buffer (a
-// last compaction when more are left), written as tokens in ascending order
+// One warp per video query block: the n_extra largest keys of its two
+// buffers (compactions when more are left), written as tokens in ascending order
 // (each lane ranks its entries by counting smaller tokens in the warp's
 // shared buffer, four per 16-byte read), -1 padded; ecnt = their count.
 constexpr int kFinThreads = 256;
@@ -476,9 +497,23 @@ __global__ void __launch_bounds__(kFinThreads) extra_finish_kernel(const SelArgs
   const int rowv = blockIdx.x * (kFinThreads / 32) + warp;   // video row over all heads
   if (rowv >= a.rows_v) return;                               // whole warp
   const int bh = rowv / a.nbv, i = a.pb + rowv % a.nbv;
-  unsigned long long* rb = a.cand + static_cast<size_t>(rowv) * kCap;
-  int count = max(0, min(__ldg(a.bcnt + rowv), kCap));
+  unsigned long long* rb = a.cand + static_cast<size_t>(rowv) * 2 * kCap;
+  unsigned long long* rb1 = rb + kCap;
   uint32_t* tok = sbuf[warp];
+  // each half's buffer down to its n_extra largest keys, the second appended
+  // to the first (2 n_extra <= kCap), then the n_extra largest of the union
+  int count = max(0, min(__ldg(a.bcnt + 2 * rowv), kCap));
+  int count1 = max(0, min(__ldg(a.bcnt + 2 * rowv + 1), kCap));
+  if (count > a.n_extra) {
+    compact_keys<kCap / 32>(rb, count, a.n_extra, reinterpret_cast<unsigned long long*>(tok));
+    count = a.n_extra;
+  }
+  if (count1 > a.n_extra) {
+    compact_keys<kCap / 32>(rb1, count1, a.n_extra, reinterpret_cast<unsigned long long*>(tok));
+    count1 = a.n_extra;
+  }
+  for (int p = lane; p < count1; p += 32) rb[count + p] = rb1[p];
+  count += count1;
   if (count > a.n_extra) {
     compact_keys<kCap / 32>(rb, count, a.n_extra, reinterpret_cast<unsigned long long*>(tok));
     count = a.n_extra;
@@ -742,8 +777,8 @@ int extra_cand_cap(int n_extra) { return n_extra <= 256 ? 768 : 2048; }
 
 size_t select_extra_scratch_bytes(const Shape& s, int n_extra) {
   if (n_extra <= 0) return 0;
-  const size_t rows = static_cast<size_t>(s.B) * s.H * s.nbv;
-  return rows * extra_cand_cap(n_extra) * 8 + rows * 4;   // buffers, then their fill counts
+  const size_t bufs = static_cast<size_t>(s.B) * s.H * s.nbv * 2;   // two per video query block
+  return bufs * extra_cand_cap(n_extra) * 8 + bufs * 4;   // buffers, then their fill counts
 }
 
 int extra_side_cap(const Shape& s, int n_extra) {
@@ -762,7 +797,8 @@ cudaError_t launch_select_extra(const Shape& s, int n_extra, const CUtensorMap& 
   a.cand = static_cast<unsigned long long*>(scratch);
   a.rows_v = s.B * s.H * s.nbv;
   a.bcnt = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) +
-                                      static_cast<size_t>(a.rows_v) * extra_cand_cap(n_extra) * 8);
+                                      static_cast<size_t>(a.rows_v) * 2 *
+                                          extra_cand_cap(n_extra) * 8);
   a.extra = extra;
   a.ecnt = ecnt;
   a.dev_status = s.dev_status;

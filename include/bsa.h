@@ -438,8 +438,9 @@ int bsa_summarize_stats(const bsa_params* p, const void* K, const void* V, const
                         float* kpool, void* ksum, void* vsum, float* bias, float* kstat,
                         float* vstat, float* lse_blk, void* stream);
 
-/* Scratch of bsa_select_extra: one candidate buffer per video query block
- * (0 for n_extra = 0); 0 also for invalid arguments. */
+/* Scratch of bsa_select_extra: two candidate buffers per video query block,
+ * one per half of each key block's tokens (0 for n_extra = 0); 0 also for
+ * invalid arguments. */
 size_t bsa_select_extra_workspace_bytes(const bsa_params* p, int32_t n_extra);
 
 /* Extra tokens of every query block.  qpool as bsa_pool wrote it, K bf16

@@ -229,8 +229,9 @@ def test_threshold_arguments_rejected_before_launch():
 
 
 def test_extra_token_sizes():
-    # side rows: min(n_extra, nbv) rounded up to 128; candidate buffers of 768
-    # keys per video query block up to 256 extra tokens, 2048 above
+    # side rows: min(n_extra, nbv) rounded up to 128; two candidate buffers
+    # (token halves) of 768 keys per video query block up to 256 extra
+    # tokens, 2048 above
     p = _p()
     bh, nb = 56, 295
     assert bsa.bsa_extra_side_capacity(p, 256) == 256
@@ -238,16 +239,15 @@ def test_extra_token_sizes():
     assert bsa.bsa_extra_side_capacity(p, 0) == 0
     assert bsa.bsa_extra_side_capacity(bsa.params(1, 1, 1000, 3), 300) == 128   # nbv = 8
     assert bsa.bsa_extra_side_capacity(p, 513) == -1 and bsa.bsa_extra_side_capacity(p, -1) == -1
-    assert bsa.bsa_select_extra_workspace_bytes(p, 256) == bh * nb * (768 * 8 + 4)
-    assert bsa.bsa_select_extra_workspace_bytes(p, 257) == bh * nb * (2048 * 8 + 4)
-    assert bsa.bsa_select_extra_workspace_bytes(p, 257) == bh * nb * (2048 * 8 + 4)
+    assert bsa.bsa_select_extra_workspace_bytes(p, 256) == 2 * bh * nb * (768 * 8 + 4)
+    assert bsa.bsa_select_extra_workspace_bytes(p, 257) == 2 * bh * nb * (2048 * 8 + 4)
     assert bsa.bsa_select_extra_workspace_bytes(p, 0) == 0
     r256 = lambda x: (x + 255) // 256 * 256
     blocks = bh * nb
     want = sum(r256(x) for x in (blocks * 512, blocks * 512, blocks * 4, blocks * 256 * 4,
                                  blocks * 4, blocks * 256 * 256, blocks * 256 * 256,
                                  blocks * 256 * 4, blocks * 256 * 4, blocks * 4,
-                                 blocks * (768 * 8 + 4)))
+                                 2 * blocks * (768 * 8 + 4)))
     assert bsa.bsa_forward_extra_workspace_bytes(p, 256) == bsa.bsa_workspace_bytes(p) + want
     # the row gathers use 32-bit row coordinates
     assert bsa.bsa_forward_extra_workspace_bytes(bsa.params(64, 16, 1 << 21, 64), 256) == 0
