@@ -18,8 +18,8 @@ its roofline peak is the measured bf16 peak times the nominal e4m3/bf16
 tensor ratio (2).  ``--tau T`` times the threshold-selection option: the
 selection keeps the key blocks at least T standard deviations above each
 row's mean score (bsa_select_threshold) and the attention runs over those
-variable-length lists (bsa_attend_lists, schedule kernels included in its
-stage time).  ``--extra-tokens N`` times the extra-token option: the N
+variable-length lists (bsa_attend_lists, its schedule kernel included in
+the stage time).  ``--extra-tokens N`` times the extra-token option: the N
 top-scoring tokens of the unlisted blocks of every query block are read
 exactly (bsa_select_extra), the blocks that lose tokens get summary rows of
 their remaining tokens (bsa_extra_summaries) and the attention reads both
@@ -756,8 +756,12 @@ def main():
                              "bytes_per_call": pool_bytes},
             "cpu_baseline": cpu,
             "e2e": e2e,
+            # per step: pool_q, anchor, summarize, select, attend; fp8 adds five
+            # quantisations and the value-scale reduction, the threshold path
+            # the schedule, the extra-token path the token selection, its
+            # finishing pass and the side summaries
             "gpu_launches": ((11 if fp8 else (6 if thr else
-                                              (5 + (2 if args.extra_tokens else 0) if xtr else 5)))
+                                              (5 + (3 if args.extra_tokens else 0) if xtr else 5)))
                              + (reblock_launches(N, prefix) + 1 if rbl else 0)) * args.steps,
             "clocks": clock_info,
             "context": {"pages_rtx_pro_6000_sparse_ms": 30.7 if cfg["N"] == 37_740 else None},
